@@ -1,0 +1,309 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+None of these retypes the oracle's formula: each checks it against an
+independent definition (brute-force dense attention, pure-Python sorting),
+a closed form, an invariance, or a convergence rate.  Every pin is built so a
+plausible slip (a dropped term, a wrong sign, index or scale, a transposed
+operand) fails at least one test.
+"""
+
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+
+RNG = np.random.default_rng(12345)
+
+
+def _rand(L, d, scale=1.0, rng=RNG):
+    return scale * rng.standard_normal((L, d))
+
+
+# ---------------------------------------------------------------- special cases
+
+
+@pytest.mark.parametrize("L,B,d", [(1000, 128, 64), (300, 64, 32), (257, 16, 8), (64, 64, 16)])
+def test_every_block_selected_equals_dense(L, B, d):
+    """k = nb (no unselected block): PISA is plain softmax attention."""
+    rng = np.random.default_rng(L + B + d)
+    q, k, v = _rand(L, d, 1.0, rng), _rand(L, d, 1.0, rng), _rand(L, d, 1.0, rng)
+    nb = -(-L // B)
+    r = oracle.pisa_head(q, k, v, B, nb)
+    ref = oracle.dense_attention(q, k, v)
+    err = np.abs(r["out"] - ref).max() / np.abs(ref).max()
+    assert err < 1e-12
+
+
+def test_single_block_equals_dense():
+    """L <= B: one block, k = 1."""
+    q, k, v = _rand(50, 16), _rand(50, 16), _rand(50, 16)
+    r = oracle.pisa_head(q, k, v, 64, 1)
+    assert r["sel"].shape == (1, 1)
+    np.testing.assert_allclose(r["out"], oracle.dense_attention(q, k, v), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("kk", [1, 2, 5])
+@pytest.mark.parametrize("L,B", [(256, 32), (250, 32)])
+def test_constant_keys_per_block_exact_for_any_k(L, B, kk):
+    """Keys constant inside every block: H_j = 0, and the zeroth-order term is
+    exact, so PISA equals dense attention whatever the selection."""
+    rng = np.random.default_rng(7 * L + kk)
+    d = 16
+    nb = -(-L // B)
+    centres = rng.standard_normal((nb, d)) * 2.0
+    k = centres[np.arange(L) // B]
+    q, v = rng.standard_normal((L, d)) * 2.0, rng.standard_normal((L, d))
+    r = oracle.pisa_head(q, k, v, B, kk)
+    assert np.abs(r["H"]).max() < 1e-12
+    np.testing.assert_allclose(r["out"], oracle.dense_attention(q, k, v), rtol=0, atol=1e-12)
+
+
+def test_zeroth_order_exact_on_a_constant_key_block():
+    """For one block whose keys all equal kbar_j: sum_n e^{s q k_n} v_n =
+    alpha * sigma_j and sum_n e^{s q k_n} = n_j * alpha."""
+    rng = np.random.default_rng(3)
+    d, n = 16, 37
+    s = 1 / math.sqrt(d)
+    key = rng.standard_normal(d)
+    kblock = np.tile(key, (n, 1))
+    vblock = rng.standard_normal((n, d))
+    q = rng.standard_normal(d)
+    _, kbar, vsum, nn = oracle.block_stats(kblock, kblock, vblock, 64)
+    alpha = math.exp(s * q @ kbar[0])
+    exact_num = sum(math.exp(s * q @ kblock[t]) * vblock[t] for t in range(n))
+    exact_den = sum(math.exp(s * q @ kblock[t]) for t in range(n))
+    np.testing.assert_allclose(alpha * vsum[0], exact_num, rtol=1e-13)
+    assert abs(nn[0] * alpha - exact_den) < 1e-12 * exact_den
+
+
+# ---------------------------------------------------------------- invariants
+
+
+def _case(L=600, B=64, d=32, seed=0):
+    rng = np.random.default_rng(seed)
+    pos = np.cumsum(rng.standard_normal((L, d)) * 0.15, axis=0)
+    q = rng.standard_normal((L, d)) + pos
+    k = rng.standard_normal((L, d)) + pos
+    v = rng.standard_normal((L, d))
+    return q, k, v
+
+
+def test_denominator_positive_and_above_exact_part():
+    q, k, v = _case()
+    r = oracle.pisa_head(q, k, v, 64, 3)
+    out, D, exact = oracle.pisa_rows(q, k, v, 64, r["sel"], r["kbar"], r["vsum"], r["n"],
+                                     r["Hbar"], np.arange(q.shape[0]), r["s"], return_parts=True)
+    assert np.all(D > 0)
+    assert np.all(D >= exact)
+    assert np.all(D > exact)  # every row has unselected blocks here
+
+
+def test_value_shift_moves_output_by_the_shift():
+    """o(V + 1c^T) = o(V) + c; H_j (hence M, S) is unchanged since the centred
+    keys sum to zero."""
+    q, k, v = _case(seed=1)
+    c = np.linspace(-2, 3, v.shape[1])
+    a = oracle.pisa_head(q, k, v, 64, 3)
+    b = oracle.pisa_head(q, k, v + c[None, :], 64, 3)
+    np.testing.assert_array_equal(a["sel"], b["sel"])
+    np.testing.assert_allclose(b["H"], a["H"], rtol=0, atol=1e-9)
+    np.testing.assert_allclose(b["out"], a["out"] + c[None, :], rtol=0, atol=1e-11)
+
+
+def test_key_shift_leaves_output_unchanged():
+    """o(K + 1c^T) = o(K): every exponent of a row moves by s q_t.c; routing
+    scores move by a per-row constant."""
+    q, k, v = _case(seed=2)
+    c = np.linspace(1, -1, k.shape[1])
+    a = oracle.pisa_head(q, k, v, 64, 3)
+    b = oracle.pisa_head(q, k + c[None, :], v, 64, 3)
+    np.testing.assert_array_equal(a["sel"], b["sel"])
+    np.testing.assert_allclose(b["M"], a["M"], rtol=1e-12)
+    diff = b["scores"] - a["scores"]
+    np.testing.assert_allclose(diff, diff[:, :1] * np.ones_like(diff), rtol=0, atol=1e-10)
+    np.testing.assert_allclose(b["out"], a["out"], rtol=0, atol=1e-11)
+
+
+def test_permutation_inside_blocks_is_invisible():
+    """Permuting tokens inside each block (same permutation for K and V) keeps
+    kbar, sigma, H, M, S and the output."""
+    q, k, v = _case(L=640, seed=3)
+    B = 64
+    rng = np.random.default_rng(9)
+    perm = np.concatenate([j * B + rng.permutation(B) for j in range(640 // B)])
+    a = oracle.pisa_head(q, k, v, B, 4)
+    b = oracle.pisa_head(q, k[perm], v[perm], B, 4)
+    np.testing.assert_array_equal(a["sel"], b["sel"])
+    np.testing.assert_allclose(b["H"], a["H"], rtol=0, atol=1e-10)
+    np.testing.assert_allclose(b["out"], a["out"], rtol=0, atol=1e-11)
+
+
+# ---------------------------------------------------------------- first-order term
+
+
+def _taylor_case(eps, shared, seed=4, L=96, B=12, d=8):
+    """Keys k_n = c_j + eps*delta_{n mod B}.  With ``shared`` the values repeat
+    the same pattern in every block, which makes every H_j equal to Hbar."""
+    rng = np.random.default_rng(seed)
+    nb = L // B
+    centres = rng.standard_normal((nb, d)) * 1.5
+    delta = rng.standard_normal((B, d))
+    k = centres[np.arange(L) // B] + eps * delta[np.arange(L) % B]
+    if shared:
+        v = rng.standard_normal((B, d))[np.arange(L) % B]
+    else:
+        v = rng.standard_normal((L, d))
+    q = rng.standard_normal((L, d)) * 1.5
+    return q, k, v
+
+
+def _pisa_fixed_sel(q, k, v, B, sel, zero_hbar=False):
+    s = 1 / math.sqrt(q.shape[1])
+    qbar, kbar, vsum, n = oracle.block_stats(q, k, v, B)
+    H = oracle.first_order_blocks(k, v, B, kbar)
+    Hbar = oracle.hbar_mean(H)
+    if zero_hbar:
+        Hbar = np.zeros_like(Hbar)
+    return oracle.pisa_rows(q, k, v, B, sel, kbar, vsum, n, Hbar, np.arange(q.shape[0]), s)
+
+
+def _slope(shared, zero_hbar):
+    B = 12
+    sel = np.array([[i, (i + 3) % 8] for i in range(8)])
+    sel.sort(axis=1)
+    eps = np.array([1e-1, 3e-2, 1e-2, 3e-3, 1e-3])
+    errs = []
+    for e in eps:
+        q, k, v = _taylor_case(e, shared)
+        errs.append(np.abs(_pisa_fixed_sel(q, k, v, B, sel, zero_hbar) - oracle.dense_attention(q, k, v)).max())
+    return np.polyfit(np.log(eps), np.log(errs), 1)[0]
+
+
+def test_first_order_term_is_second_order_exact_when_blocks_share_structure():
+    """All H_j equal Hbar: the hybrid first-order term is the block's own
+    first-order Taylor term, so the error is O(eps^2)."""
+    assert _slope(shared=True, zero_hbar=False) == pytest.approx(2.0, abs=0.15)
+
+
+def test_dropping_the_first_order_term_leaves_first_order_error():
+    """Same inputs with Hbar removed (a planted slip): the error is O(eps)."""
+    assert _slope(shared=True, zero_hbar=True) == pytest.approx(1.0, abs=0.15)
+
+
+def test_hybrid_error_is_first_order_for_generic_blocks():
+    """Different H_j per block: Hbar only captures their mean, error O(eps)."""
+    assert _slope(shared=False, zero_hbar=False) == pytest.approx(1.0, abs=0.15)
+
+
+def test_first_order_matrix_identity():
+    """H_j = K_j^T V_j - n_j kbar_j^T vbar_j, and sum_j H_j = K^T V - sum_j n_j kbar_j^T vbar_j."""
+    q, k, v = _case(L=650, seed=5)
+    B = 64
+    qbar, kbar, vsum, n = oracle.block_stats(q, k, v, B)
+    H = oracle.first_order_blocks(k, v, B, kbar)
+    total = np.zeros_like(H[0])
+    for j in range(len(n)):
+        a, b = j * B, min((j + 1) * B, 650)
+        alt = k[a:b].T @ v[a:b] - np.outer(kbar[j], vsum[j])
+        np.testing.assert_allclose(H[j], alt, rtol=0, atol=1e-10)
+        total += np.outer(kbar[j], vsum[j])
+    np.testing.assert_allclose(H.sum(axis=0), k.T @ v - total, rtol=0, atol=1e-9)
+    np.testing.assert_allclose(oracle.hbar_mean(H), H.sum(axis=0) / len(n), rtol=1e-14)
+
+
+# ---------------------------------------------------------------- routing
+
+
+def test_covariance_norm_closed_form():
+    """H_j = lambda_j * c * e_1 w^T (only coordinate 0 of the keys varies inside
+    a block, values lambda_j delta_n w): M_j = |lambda_j - mean(lambda)| c ||w||."""
+    rng = np.random.default_rng(6)
+    B, nb, d = 16, 6, 8
+    delta = rng.standard_normal(B)
+    delta -= delta.mean()
+    lam = rng.standard_normal(nb)
+    w = rng.standard_normal(d)
+    centres = rng.standard_normal((nb, d))
+    k = np.zeros((nb * B, d))
+    v = np.zeros((nb * B, d))
+    for j in range(nb):
+        k[j * B:(j + 1) * B] = centres[j]
+        k[j * B:(j + 1) * B, 0] += delta
+        v[j * B:(j + 1) * B] = lam[j] * delta[:, None] * w[None, :]
+    _, kbar, _, _ = oracle.block_stats(k, k, v, B)
+    H = oracle.first_order_blocks(k, v, B, kbar)
+    M = oracle.cov_norm(H, oracle.hbar_mean(H))
+    c = (delta ** 2).sum()
+    np.testing.assert_allclose(M, np.abs(lam - lam.mean()) * c * np.linalg.norm(w), rtol=1e-12)
+
+
+def _brute_topk_pooled(q, k, B, kk):
+    """Pure-Python pooled block-sparse routing: block means, scaled dot plus
+    ln(block size), full sort with ties to the smaller index."""
+    L, d = len(q), len(q[0])
+    nb = -(-L // B)
+    s = 1 / math.sqrt(d)
+    means = []
+    for X in (q, k):
+        mm = []
+        for j in range(nb):
+            rows = X[j * B:min((j + 1) * B, L)]
+            mm.append([sum(r[a] for r in rows) / len(rows) for a in range(d)])
+        means.append(mm)
+    sizes = [min((j + 1) * B, L) - j * B for j in range(nb)]
+    sel, gaps = [], []
+    for i in range(nb):
+        sc = [(s * sum(means[0][i][a] * means[1][j][a] for a in range(d)) + math.log(sizes[j]), j)
+              for j in range(nb)]
+        ranked = sorted(sc, key=lambda t: (-t[0], t[1]))
+        sel.append(sorted(j for _, j in ranked[:kk]))
+        if kk < nb:
+            gaps.append(ranked[kk - 1][0] - ranked[kk][0])
+    return sel, min(gaps)
+
+
+@pytest.mark.parametrize("L,B,kk", [(500, 50, 3), (470, 50, 4), (256, 32, 1)])
+def test_zero_values_reduce_routing_to_pooled_topk(L, B, kk):
+    """V = 0: every H_j = 0, M = 0, and the score is textbook pooled block
+    routing s qbar.kbar + ln n_j (brute force, pure Python)."""
+    q, k, _ = _case(L=L, B=B, d=12, seed=L + kk)
+    v = np.zeros_like(q)
+    r = oracle.pisa_head(q, k, v, B, kk)
+    assert np.abs(r["M"]).max() == 0.0
+    sel, gap = _brute_topk_pooled(q.tolist(), k.tolist(), B, kk)
+    assert gap > 1e-9
+    np.testing.assert_array_equal(r["sel"], np.array(sel))
+
+
+def test_topk_ties_go_to_the_smaller_index():
+    scores = np.array([[1.0, 3.0, 3.0, 2.0, 3.0],
+                       [0.0, 0.0, 0.0, 0.0, 0.0]])
+    np.testing.assert_array_equal(oracle.select_topk(scores, 2), [[1, 2], [0, 1]])
+    np.testing.assert_array_equal(oracle.select_topk(scores, 3), [[1, 2, 4], [0, 1, 2]])
+
+
+def test_scores_reduce_to_pooled_when_covariance_norm_constant():
+    """With M_j constant over j and full blocks, the ranking is the pooled one."""
+    rng = np.random.default_rng(8)
+    qbar, kbar = rng.standard_normal((10, 6)), rng.standard_normal((10, 6))
+    n = np.full(10, 32.0)
+    a = oracle.route_scores(qbar, kbar, np.full(10, 5.0), n, 0.4)
+    b = 0.4 * qbar @ kbar.T
+    np.testing.assert_array_equal(oracle.select_topk(a, 3), oracle.select_topk(b, 3))
+
+
+def test_keep_count_on_the_workloads():
+    assert oracle.keep_count(1024, 64, 4 / 16) == 4
+    assert oracle.keep_count(4608, 64, 0.25) == 18
+    assert oracle.keep_count(32760, 128, 0.15) == 39
+    assert oracle.keep_count(75600, 128, 0.10) == 60
+    assert oracle.keep_count(119040, 128, 0.08) == 75
+    assert oracle.keep_count(100, 128, 0.01) == 1
+    assert oracle.keep_count(1000, 100, 1.0) == 10
+
+
+def test_block_bounds_partial_tail():
+    s, e = oracle.block_bounds(300, 128)
+    assert s.tolist() == [0, 128, 256] and e.tolist() == [128, 256, 300]
