@@ -1,0 +1,452 @@
+"""Benchmark of the PISA piecewise sparse attention forward on B200.
+
+One step = one full forward (block stats -> covariance norm -> routing ->
+fused attention) over one batch of the named synthetic workload, inputs
+resident in HBM.  Prints ONE JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload wan720]
+    python bench.py --impl reference ...   # the fp64 CPU oracle, bounded sample
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs the same workload on
+its own GPU (weak scaling, no data-path collective); the step time is the max
+over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import config as workload_config, generate, load_redraws  # noqa: E402
+
+METRIC = "PISA attn fwd ms & effective TFLOPS at Wan-like shape; % of bf16 tensor peak"
+DEFAULT_WORKLOAD = "wan720"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def describe(cfg, kk):
+    grid = "x".join(str(g) for g in cfg.grid) if cfg.grid else "-"
+    return (f"{cfg.name}: batch {cfg.batch}, {cfg.heads} heads, L={cfg.L} ({grid}), head_dim {cfg.d}, "
+            f"block {cfg.block}, keep {cfg.keep_ratio:g} (k={kk} of {cfg.nb}), {cfg.dtype}")
+
+
+def block_sizes(cfg):
+    n = np.full(cfg.nb, cfg.block, dtype=np.int64)
+    n[-1] = cfg.L - (cfg.nb - 1) * cfg.block
+    return n
+
+
+def effective_flops(cfg, sel):
+    """Algorithmic FLOPs of one forward: exact = 4 d sum_i n_i sum_{j in S_i} n_j;
+    approx = 4 d sum_i n_i |U_i| + 2 L d^2 + L d (per batch*head, summed)."""
+    n = block_sizes(cfg).astype(np.float64)
+    d, L = cfg.d, cfg.L
+    sel = sel.reshape(-1, cfg.nb, sel.shape[-1])
+    kk = sel.shape[-1]
+    exact = 4.0 * d * float((n[None, :] * n[sel].sum(axis=-1)).sum())
+    approx_per = 4.0 * d * float(n.sum()) * (cfg.nb - kk) + 2.0 * L * d * d + L * d
+    return exact, approx_per * sel.shape[0]
+
+
+def stage_bytes(cfg, kk):
+    """Algorithmic HBM bytes per launch of the streaming kernels."""
+    bh, L, d, nb = cfg.batch * cfg.heads, cfg.L, cfg.d, cfg.nb
+    e = 2 if cfg.dtype == "bf16" else 4
+    stats = bh * (3 * L * d * e + 3 * nb * d * 4)
+    cov = bh * (2 * L * d * e + 2 * nb * d * 4 + nb * 4)
+    select = bh * (2 * nb * d * 4 + nb * 4 + nb * kk * 4)
+    return dict(stats=stats, cov_norm=cov, select=select)
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"], bf16_sustained=p["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.file.flush()
+        rows = []
+        with open(self.file.name) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.file.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def host_info():
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return model, os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+
+def oracle_step(cfg, qh, kh, vh, kk, block_stride):
+    """One bounded sample of the workload on the fp64 oracle: the whole (batch,
+    head)'s statistics and routing, then the output rows of every
+    ``block_stride``-th query block.  The statistics time is charged pro rata
+    to the rows computed.  Returns (flops, charged seconds, rows)."""
+    import oracle  # CPU baseline only: nothing else in the bench touches the oracle
+    q, k, v = (x.astype(np.float64) for x in (qh, kh, vh))
+    t0 = time.perf_counter()
+    s = 1.0 / math.sqrt(cfg.d)
+    qbar, kbar, vsum, n = oracle.block_stats(q, k, v, cfg.block)
+    H = oracle.first_order_blocks(k, v, cfg.block, kbar)
+    Hbar = oracle.hbar_mean(H)
+    M = oracle.cov_norm(H, Hbar)
+    sel = oracle.select_topk(oracle.route_scores(qbar, kbar, M, n, s), kk)
+    t1 = time.perf_counter()
+    blocks = np.arange(0, cfg.nb, block_stride)
+    rows = np.concatenate([np.arange(i * cfg.block, min((i + 1) * cfg.block, cfg.L)) for i in blocks])
+    oracle.pisa_rows(q, k, v, cfg.block, sel, kbar, vsum, n, Hbar, rows, s)
+    t2 = time.perf_counter()
+    nbk = block_sizes(cfg).astype(np.float64)
+    ex = 4.0 * cfg.d * float((nbk[blocks] * nbk[sel[blocks]].sum(axis=-1)).sum())
+    ap = 4.0 * cfg.d * float(nbk[blocks].sum()) * (cfg.nb - kk) + (2.0 * cfg.d * cfg.d + cfg.d) * len(rows)
+    charged = (t1 - t0) * len(rows) / cfg.L + (t2 - t1)
+    return ex + ap, charged, len(rows)
+
+
+def cpu_oracle_sample(cfg, q, k, v, kk, budget_s, block_stride=4):
+    """Time the oracle on successive (batch, head) samples until ``budget_s``
+    charged seconds are spent.  Returns (TFLOP/s, description, threads, seconds)."""
+    qf, kf, vf = (x.reshape(-1, cfg.L, cfg.d) for x in (q, k, v))
+    flops = spent = 0.0
+    rows = heads = 0
+    for bh in range(qf.shape[0]):
+        f, t, r = oracle_step(cfg, qf[bh], kf[bh], vf[bh], kk, block_stride)
+        flops, spent, rows, heads = flops + f, spent + t, rows + r, heads + 1
+        if spent >= budget_s:
+            break
+    desc = (f"{heads} (batch, head) slices: full statistics and routing, output rows of every "
+            f"{block_stride}th query block ({rows} rows), statistics time charged per row")
+    return flops / spent / 1e12, desc, os.cpu_count() or 1, spent
+
+
+def run_reference(args, cfg, kk):
+    """--impl reference: the fp64 oracle as it stands on the host cores; each
+    step is one bounded sample (one (batch, head), every 4th query block)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    nsl = min(cfg.batch * cfg.heads, 4)
+    table = load_redraws(cfg.name)
+    q, k, v = generate(cfg, heads=list(range(nsl)), redraws={bh: table.get(bh, {}) for bh in range(nsl)})
+    q, k, v = (x.reshape(-1, cfg.L, cfg.d) for x in (q, k, v))
+    per_step = []
+    for step in range(args.warmup + args.steps):
+        bh = step % nsl
+        t0 = time.perf_counter()
+        f, charged, rows = oracle_step(cfg, q[bh], k[bh], v[bh], kk, 4)
+        if step >= args.warmup:
+            per_step.append((f, charged))
+    flops = sum(f for f, _ in per_step)
+    spent = sum(t for _, t in per_step)
+    value = flops / spent / 1e12
+    full_flops = None
+    model, cores = host_info()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": spent / len(per_step) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": describe(cfg, kk), "parallelism": "host cores",
+                   "sample": "per step: one (batch, head), full statistics and routing, output rows of "
+                             "every 4th query block; statistics time charged per row"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": os.cpu_count() or 1, "kind": "oracle",
+                         "sample": "per step: one (batch, head), every 4th query block", "cpu": model},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU path
+
+
+def _source_sha(paths):
+    import hashlib
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu capture, or None when the
+    kernel's sources changed since the capture (or none was taken)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        table = json.load(f)
+    e = table.get(kernel, {}).get(workload)
+    if not e:
+        return None
+    try:
+        if _source_sha(e["sources"]) != e["source_sha"]:
+            return None
+    except OSError:
+        return None
+    return e["bytes_per_launch"]
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="pisa", choices=["pisa", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of oracle time for the cpu_baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    cfg = workload_config(args.workload)
+
+    if args.impl == "reference":
+        import oracle  # reference arm: the oracle as it stands
+        return run_reference(args, cfg, oracle.keep_count(cfg.L, cfg.block, cfg.keep_ratio))
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+
+    # inputs first (the generator's worker pool is spawned, before any CUDA use)
+    q, k, v = generate(cfg)
+
+    import torch
+    import sparse_attention_diffusion_block_b200 as pisa
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    kk = pisa.keep_count(cfg.L, cfg.block, cfg.keep_ratio)
+    tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    qd, kd, vd = (torch.from_numpy(x).to(dev).to(tdt) for x in (q, k, v))
+    b, h, L, d, B, nb = cfg.batch, cfg.heads, cfg.L, cfg.d, cfg.block, cfg.nb
+    f32 = dict(dtype=torch.float32, device=dev)
+    stats = (torch.empty(b, h, nb, d, **f32), torch.empty(b, h, nb, d, **f32),
+             torch.empty(b, h, nb, d, **f32), torch.empty(b, h, d, d, **f32))
+    M = torch.empty(b, h, nb, **f32)
+    sel = torch.empty(b, h, nb, kk, dtype=torch.int32, device=dev)
+    out = torch.empty_like(qd)
+    u8 = dict(dtype=torch.uint8, device=dev)
+    ws_stats = torch.empty(max(pisa.stats_workspace_size(b, h, L, d, B), 16), **u8)
+    ws_fused = torch.empty(max(pisa.fused_workspace_size(b, h, L, d, B), 16), **u8)
+    ws_all = torch.empty(pisa.workspace_size(b, h, L, d, B, kk), **u8)
+
+    def forward(ev=None):
+        if ev: ev[0].record()
+        pisa.block_stats(qd, kd, vd, B, workspace=ws_stats, out=stats)
+        if ev: ev[1].record()
+        pisa.cov_norm(kd, vd, B, stats[1], stats[2], stats[3], out=M)
+        if ev: ev[2].record()
+        pisa.select(stats[0], stats[1], M, L, B, kk, out=sel)
+        if ev: ev[3].record()
+        pisa.attn_fwd_with_sel(qd, kd, vd, B, stats[1], stats[2], stats[3], sel, out=out, workspace=ws_fused)
+        if ev: ev[4].record()
+
+    # correctness guard: the staged calls equal the one-shot entry point
+    forward()
+    ref_out = pisa.attn_fwd(qd, kd, vd, B, cfg.keep_ratio, workspace=ws_all)
+    torch.cuda.synchronize()
+    if not torch.equal(ref_out, out):
+        raise RuntimeError("staged forward differs from pisa_attn_fwd")
+    del ref_out
+    status = pisa.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {pisa.status_string(status)}")
+    sel_np = sel.cpu().numpy()
+    exact, approx = effective_flops(cfg, sel_np)
+    flops = exact + approx
+
+    for _ in range(args.warmup):
+        forward()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t0.record()
+        for s in range(K):
+            forward(evs[s])
+        t1.record()
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    total_ms = t0.elapsed_time(t1)
+    names = ["stats", "cov_norm", "select", "fused"]
+    stage_ms = {n: sum(e[i].elapsed_time(e[i + 1]) for e in evs) / K for i, n in enumerate(names)}
+    if dist:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms = total_ms / K
+    value = world * flops / (ms * 1e-3) / 1e12
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (x.to("cpu").pin_memory() for x in (qd, kd, vd))
+        oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        def e2e_step():
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            pisa.attn_fwd(qd, kd, vd, B, cfg.keep_ratio, out=out, workspace=ws_all)
+            oh.copy_(out, non_blocking=True)
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(K):
+            e2e_step()
+        z.record()
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(z)
+        if dist:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e_ms /= K
+        in_bytes = sum(x.numel() * x.element_size() for x in (qd, kd, vd))
+        e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e_ms,
+               "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out.numel() * out.element_size()}
+
+    peaks = measured_peaks()
+    fused_ms = stage_ms["fused"]
+    achieved = flops / (fused_ms * 1e-3) / 1e12
+    peak = peaks["bf16_sustained"]
+    traffic = stored_traffic("fused", cfg.name)
+    roofline = {"kernel": "fused attention (attn_fwd_with_sel)", "bound": "tensor",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": traffic,
+                "peak_source": f"{peaks['source']} sustained cuBLAS bf16 (timed inside a long step)"}
+    sbytes = stage_bytes(cfg, kk)
+    stages = {}
+    for n in names:
+        ent = {"ms": stage_ms[n]}
+        if n in sbytes:
+            gbs = sbytes[n] / (stage_ms[n] * 1e-3) / 1e9
+            ent.update({"algorithmic_bytes": sbytes[n], "GB/s": gbs, "frac_hbm": gbs / peaks["hbm"]})
+        stages[n] = ent
+    stages["fused"]["TFLOP/s"] = achieved
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, desc, threads, spent = cpu_oracle_sample(cfg, q, k, v, kk, args.cpu_budget)
+        model, _ = host_info()
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"fp64 oracle on {desc}; {spent:.1f} s", "cpu": model}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+            "config": {"workload": describe(cfg, kk), "global_batch": world * cfg.batch,
+                       "seq_len": cfg.L, "parallelism": f"replicas x{world} (one full forward per GPU)",
+                       "l2": f"inputs {3 * qd.numel() * qd.element_size() / 1e9:.2f} GB > L2 126 MB",
+                       "flops_exact": exact, "flops_approx": approx},
+            "roofline": roofline,
+            "stages": stages,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": K * pisa.LAUNCHES["attn_fwd"],
+            "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

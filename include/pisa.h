@@ -1,0 +1,158 @@
+/*
+ * pisa.h - C ABI of the B200 (sm_100a) PISA piecewise sparse attention forward.
+ *
+ * The method (gist.science technical summary of "PISA: Piecewise Sparse
+ * Attention Is Wiser for Efficient Diffusion Transformers", section 2
+ * "Method"; AI Radio episode summary of the same paper):
+ *   Q, K, V are cut into blocks of B tokens.  For query block i the KV blocks
+ *   split into a selected set S_i (exact softmax attention) and the rest U_i,
+ *   which enter the same softmax numerator N_t and denominator D_t through a
+ *   block-wise zeroth-order Taylor term (key centroid kbar_j, value sum
+ *   sigma_j) plus one global first-order correction s * beta_t * (q_t Hbar),
+ *   Hbar being the mean of the block-wise first-order matrices H_j and beta_t
+ *   the sum of the U_i weights alpha_{t,j} = exp(s q_t . kbar_j).  o_t = N_t/D_t.
+ *   S_i is the top-k of a covariance-aware score that uses M_j = ||H_j - Hbar||.
+ *
+ * Conventions shared by every entry point:
+ *   - Tensors are dense row-major.  q, k, v, out: [batch, heads, L, d]
+ *     (element type given by `dtype`; out has the input type).  Per-block
+ *     statistics: [batch, heads, nb, d] float32 with nb = ceil(L / block);
+ *     Hbar: [batch, heads, d, d] float32 (row = key dimension, column = value
+ *     dimension); M: [batch, heads, nb] float32; sel: [batch, heads, nb, k]
+ *     int32, each row ascending.
+ *   - All pointers except `stream` are DEVICE pointers owned by the caller,
+ *     16-byte aligned.  The library never allocates device memory; scratch
+ *     space comes from the caller's `workspace` (size from the *_workspace_size
+ *     query).  `stream` is a cudaStream_t passed as void* (NULL = legacy default).
+ *   - Calls are asynchronous on `stream`.  Arguments are validated on the host
+ *     before any launch; a rejected call launches nothing and returns an error.
+ *     Launch failures return PISA_ERR_CUDA.  Device-side checks (bounded waits,
+ *     index checks) record an error word read by pisa_device_status().
+ *   - Supported: d in {64, 128}, block in {64, 128}, 1 <= L, 1 <= k <= nb,
+ *     batch*heads >= 1.  The softmax scale is fixed at 1/sqrt(d).
+ *   - Reading of the pages used throughout: scores carry the scale s=1/sqrt(d)
+ *     (also inside the first-order term); H_j = sum_n (k_n - kbar_j)^T v_n (a
+ *     sum, d x d); Hbar is the plain mean of H_j over all nb blocks of the
+ *     (batch, head); beta_t = sum_{j in U_i} alpha_{t,j}; the norm in M_j is
+ *     Frobenius; a partial last block keeps its true size n_j.
+ */
+#ifndef PISA_H
+#define PISA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pisa_status {
+  PISA_OK = 0,
+  PISA_ERR_INVALID_ARG = -1,  /* null pointer, bad size, misaligned pointer */
+  PISA_ERR_UNSUPPORTED = -2,  /* d or block outside the supported set      */
+  PISA_ERR_WORKSPACE = -3,    /* workspace missing or smaller than needed  */
+  PISA_ERR_CUDA = -4,         /* a CUDA runtime call or launch failed      */
+  PISA_ERR_TIMEOUT = -5,      /* a bounded device wait ran out             */
+  PISA_ERR_DEVICE_CHECK = -6  /* a device-side index check failed          */
+} pisa_status;
+
+typedef enum pisa_dtype {
+  PISA_BF16 = 0,
+  PISA_FP32 = 1
+} pisa_dtype;
+
+/* Text of a status code (static storage, never NULL). */
+const char* pisa_status_string(pisa_status status);
+
+/* Number of exactly computed KV blocks per query block for a keep ratio rho:
+ * k = clamp(ceil(rho * nb - 1e-9), 1, nb), nb = ceil(L / block), computed in
+ * double from the float argument.  Returns -1 for L < 1, block < 1 or a
+ * non-finite / non-positive rho. */
+int pisa_keep_count(int L, int block, float keep_ratio);
+
+/* Scratch bytes pisa_block_stats needs (per-chunk partial sums of H_j). */
+size_t pisa_stats_workspace_size(int batch, int heads, int L, int d, int block);
+
+/* Scratch bytes pisa_attn_fwd_with_sel needs (centroid and Hbar operands in
+ * the fused kernel's input format). */
+size_t pisa_fused_workspace_size(int batch, int heads, int L, int d, int block);
+
+/* Scratch bytes pisa_attn_fwd needs for all stages with k selected blocks. */
+size_t pisa_workspace_size(int batch, int heads, int L, int d, int block, int k);
+
+/* Block statistics (gist.science summary, section 2, hardware implementation:
+ * the precompute of block centroids, value sums and Hbar).
+ *   qbar[i] = mean of the query rows of block i   (pooled query, routing only)
+ *   kbar[j] = mean of the key rows of block j      (centroid)
+ *   vsum[j] = sum of the value rows of block j     (sigma_j)
+ *   hbar    = (1/nb) sum_j H_j,  H_j = sum_n (k_n - kbar_j)^T v_n
+ * Reads q, k, v once.  hbar is reduced in a fixed order (no float atomics), so
+ * results are bit-reproducible.  workspace >= pisa_stats_workspace_size(). */
+pisa_status pisa_block_stats(const void* q, const void* k, const void* v, pisa_dtype dtype,
+                             int batch, int heads, int L, int d, int block,
+                             float* qbar, float* kbar, float* vsum, float* hbar,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Covariance norm for routing (gist.science summary, section 2,
+ * covariance-aware routing): M[j] = ||H_j - Hbar||_F, recomputing each H_j from
+ * k, v and the stats of pisa_block_stats instead of storing all of them. */
+pisa_status pisa_cov_norm(const void* k, const void* v, pisa_dtype dtype,
+                          int batch, int heads, int L, int d, int block,
+                          const float* kbar, const float* vsum, const float* hbar,
+                          float* M, void* stream);
+
+/* Block-wise first-order matrices H_j, written out: H [batch, heads, nb, d, d]
+ * float32.  Not on the attention path (which never stores them); for
+ * inspection and tests. */
+pisa_status pisa_block_first_order(const void* k, const void* v, pisa_dtype dtype,
+                                   int batch, int heads, int L, int d, int block,
+                                   const float* kbar, const float* vsum, float* H,
+                                   void* stream);
+
+/* Covariance-aware top-k routing (AI Radio summary: Score_{t,j}; gist.science
+ * summary, section 2, covariance-aware routing).  Score of KV block j for
+ * query block i:
+ *     score = s * qbar_i . kbar_j + ln(n_j + s * ||qbar_i||_2 * M_j)
+ * (reading: log of the block's zeroth-order mass times its size plus the
+ * Cauchy-Schwarz bound of the first-order error left by Hbar).  sel[i] = the k
+ * largest scores, exact ties to the smaller j, stored ascending.  Scores are
+ * float32. */
+pisa_status pisa_select(const float* qbar, const float* kbar, const float* M,
+                        int batch, int heads, int L, int d, int block, int k,
+                        int32_t* sel, void* stream);
+
+/* The fused forward for a given selection (gist.science summary, section 2:
+ * core algorithm, N_t equation; hardware implementation phases 1-3).  For
+ * every query row t of block i, in one online softmax:
+ *   exact:  x = s q_t . k_n for the tokens of the blocks in sel[i]
+ *   approx: y = s q_t . kbar_j for the other blocks, weight e^y, mass n_j e^y,
+ *           value sum vsum_j, beta_t += e^y
+ *   out_t = (sum e^x v_n + sum e^y vsum_j + s beta_t (q_t hbar))
+ *           / (sum e^x + sum n_j e^y)
+ * kbar, vsum, hbar as produced by pisa_block_stats; sel as produced by
+ * pisa_select (entries in [0, nb), ascending, no repeats).
+ * workspace >= pisa_fused_workspace_size(). */
+pisa_status pisa_attn_fwd_with_sel(const void* q, const void* k, const void* v, void* out,
+                                   pisa_dtype dtype, int batch, int heads, int L, int d,
+                                   int block, const float* kbar, const float* vsum,
+                                   const float* hbar, const int32_t* sel, int k_sel,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* The whole forward: block stats -> covariance norm -> routing -> fused
+ * attention, with k = pisa_keep_count(L, block, keep_ratio).
+ * workspace >= pisa_workspace_size(batch, heads, L, d, block, k). */
+pisa_status pisa_attn_fwd(const void* q, const void* k, const void* v, void* out,
+                          pisa_dtype dtype, int batch, int heads, int L, int d, int block,
+                          float keep_ratio, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/* Reads (and, when reset != 0, clears) the device error word that bounded
+ * waits and index checks set.  Synchronises `stream`.  Returns PISA_OK,
+ * PISA_ERR_TIMEOUT, PISA_ERR_DEVICE_CHECK or PISA_ERR_CUDA. */
+pisa_status pisa_device_status(void* stream, int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PISA_H */

@@ -1,0 +1,226 @@
+"""Python binding of libpisa.so, the B200 PISA piecewise sparse attention library.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in include/pisa.h.  PyTorch provides device
+memory and streams.  There is no CPU fallback: importing this module fails
+loudly when the library has not been built.
+
+Entry points mirror the C names (without the ``pisa_`` prefix):
+block_stats, cov_norm, block_first_order, select, attn_fwd_with_sel, attn_fwd,
+keep_count, workspace_size, stats_workspace_size, fused_workspace_size,
+device_status, status_string.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpisa.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m sparse_attention_diffusion_block_b200.build` "
+        "(nvcc, sm_100a).  There is no fallback implementation.")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+PISA_OK = 0
+PISA_ERR_INVALID_ARG = -1
+PISA_ERR_UNSUPPORTED = -2
+PISA_ERR_WORKSPACE = -3
+PISA_ERR_CUDA = -4
+PISA_ERR_TIMEOUT = -5
+PISA_ERR_DEVICE_CHECK = -6
+PISA_BF16 = 0
+PISA_FP32 = 1
+
+EXPORTS = (
+    "pisa_status_string", "pisa_keep_count", "pisa_stats_workspace_size",
+    "pisa_fused_workspace_size", "pisa_workspace_size", "pisa_block_stats", "pisa_cov_norm",
+    "pisa_block_first_order", "pisa_select", "pisa_attn_fwd_with_sel", "pisa_attn_fwd",
+    "pisa_device_status",
+)
+
+_p = ctypes.c_void_p
+_i = ctypes.c_int
+_z = ctypes.c_size_t
+_f = ctypes.c_float
+
+
+def _sig(name, restype, *argtypes):
+    fn = getattr(_lib, name)
+    fn.restype = restype
+    fn.argtypes = list(argtypes)
+    return fn
+
+
+_lib_status_string = _sig("pisa_status_string", ctypes.c_char_p, _i)
+_lib_keep_count = _sig("pisa_keep_count", _i, _i, _i, _f)
+_lib_stats_ws = _sig("pisa_stats_workspace_size", _z, _i, _i, _i, _i, _i)
+_lib_fused_ws = _sig("pisa_fused_workspace_size", _z, _i, _i, _i, _i, _i)
+_lib_ws = _sig("pisa_workspace_size", _z, _i, _i, _i, _i, _i, _i)
+_lib_block_stats = _sig("pisa_block_stats", _i, _p, _p, _p, _i, _i, _i, _i, _i, _i,
+                        _p, _p, _p, _p, _p, _z, _p)
+_lib_cov_norm = _sig("pisa_cov_norm", _i, _p, _p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p)
+_lib_first_order = _sig("pisa_block_first_order", _i, _p, _p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p)
+_lib_select = _sig("pisa_select", _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p, _p)
+_lib_fwd_sel = _sig("pisa_attn_fwd_with_sel", _i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i,
+                    _p, _p, _p, _p, _i, _p, _z, _p)
+_lib_fwd = _sig("pisa_attn_fwd", _i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p, _z, _p)
+_lib_device_status = _sig("pisa_device_status", _i, _p, _i)
+
+
+class PisaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {status_string(code)} ({code})")
+        self.code = code
+
+
+def raw_lib() -> ctypes.CDLL:
+    """The loaded ctypes library (for tests of the raw C ABI)."""
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return _lib_status_string(int(code)).decode()
+
+
+def _check(code: int, where: str) -> None:
+    if code != PISA_OK:
+        raise PisaError(code, where)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return PISA_BF16
+    if t.dtype == torch.float32:
+        return PISA_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}: bf16 or fp32")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _qkv_shape(q: torch.Tensor):
+    if q.dim() != 4:
+        raise ValueError("q, k, v must be [batch, heads, L, d]")
+    b, h, L, d = q.shape
+    return b, h, L, d
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def keep_count(L: int, block: int, keep_ratio: float) -> int:
+    return int(_lib_keep_count(int(L), int(block), float(keep_ratio)))
+
+
+def stats_workspace_size(batch, heads, L, d, block) -> int:
+    return int(_lib_stats_ws(batch, heads, L, d, block))
+
+
+def fused_workspace_size(batch, heads, L, d, block) -> int:
+    return int(_lib_fused_ws(batch, heads, L, d, block))
+
+
+def workspace_size(batch, heads, L, d, block, k) -> int:
+    return int(_lib_ws(batch, heads, L, d, block, k))
+
+
+def _workspace(nbytes: int, device, given: Optional[torch.Tensor]):
+    if given is not None:
+        return given
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+def block_stats(q, k, v, block, workspace=None, stream=None, out=None):
+    """(qbar, kbar, vsum, hbar) float32 for [b,h,L,d] inputs (``out``: the four
+    tensors, preallocated)."""
+    _need_cuda(q, k, v)
+    b, h, L, d = _qkv_shape(q)
+    nb = -(-L // block)
+    f = dict(dtype=torch.float32, device=q.device)
+    if out is None:
+        out = (torch.empty(b, h, nb, d, **f), torch.empty(b, h, nb, d, **f),
+               torch.empty(b, h, nb, d, **f), torch.empty(b, h, d, d, **f))
+    qbar, kbar, vsum, hbar = out
+    ws = _workspace(stats_workspace_size(b, h, L, d, block), q.device, workspace)
+    _check(_lib_block_stats(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), b, h, L, d, block,
+                            _ptr(qbar), _ptr(kbar), _ptr(vsum), _ptr(hbar), _ptr(ws), ws.numel(),
+                            _stream(stream)), "pisa_block_stats")
+    return qbar, kbar, vsum, hbar
+
+
+def cov_norm(k, v, block, kbar, vsum, hbar, stream=None, out=None):
+    _need_cuda(k, v, kbar, vsum, hbar)
+    b, h, L, d = _qkv_shape(k)
+    M = out if out is not None else torch.empty(b, h, -(-L // block), dtype=torch.float32, device=k.device)
+    _check(_lib_cov_norm(_ptr(k), _ptr(v), _dtype_code(k), b, h, L, d, block, _ptr(kbar), _ptr(vsum),
+                         _ptr(hbar), _ptr(M), _stream(stream)), "pisa_cov_norm")
+    return M
+
+
+def block_first_order(k, v, block, kbar, vsum, stream=None):
+    _need_cuda(k, v, kbar, vsum)
+    b, h, L, d = _qkv_shape(k)
+    H = torch.empty(b, h, -(-L // block), d, d, dtype=torch.float32, device=k.device)
+    _check(_lib_first_order(_ptr(k), _ptr(v), _dtype_code(k), b, h, L, d, block, _ptr(kbar),
+                            _ptr(vsum), _ptr(H), _stream(stream)), "pisa_block_first_order")
+    return H
+
+
+def select(qbar, kbar, M, L, block, k, stream=None, out=None):
+    _need_cuda(qbar, kbar, M)
+    b, h, nb, d = qbar.shape
+    sel = out if out is not None else torch.empty(b, h, nb, k, dtype=torch.int32, device=qbar.device)
+    _check(_lib_select(_ptr(qbar), _ptr(kbar), _ptr(M), b, h, L, d, block, k, _ptr(sel),
+                       _stream(stream)), "pisa_select")
+    return sel
+
+
+def attn_fwd_with_sel(q, k, v, block, kbar, vsum, hbar, sel, out=None, workspace=None, stream=None):
+    _need_cuda(q, k, v, kbar, vsum, hbar, sel)
+    b, h, L, d = _qkv_shape(q)
+    if out is None:
+        out = torch.empty_like(q)
+    ws = _workspace(fused_workspace_size(b, h, L, d, block), q.device, workspace)
+    _check(_lib_fwd_sel(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), b, h, L, d, block,
+                        _ptr(kbar), _ptr(vsum), _ptr(hbar), _ptr(sel), int(sel.shape[-1]), _ptr(ws),
+                        ws.numel(), _stream(stream)), "pisa_attn_fwd_with_sel")
+    return out
+
+
+def attn_fwd(q, k, v, block, keep_ratio, out=None, workspace=None, stream=None):
+    """PISA forward: out [b,h,L,d] with the dtype of q."""
+    _need_cuda(q, k, v)
+    b, h, L, d = _qkv_shape(q)
+    if out is None:
+        out = torch.empty_like(q)
+    kk = keep_count(L, block, keep_ratio)
+    ws = _workspace(workspace_size(b, h, L, d, block, kk), q.device, workspace)
+    _check(_lib_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), b, h, L, d, block,
+                    float(keep_ratio), _ptr(ws), ws.numel(), _stream(stream)), "pisa_attn_fwd")
+    return out
+
+
+# Kernels each entry point launches (for launch accounting in the bench).
+LAUNCHES = {"block_stats": 2, "cov_norm": 1, "select": 1, "attn_fwd_with_sel": 1}
+LAUNCHES["attn_fwd"] = sum(LAUNCHES.values())
+
+
+def device_status(stream=None, reset: bool = True) -> int:
+    return int(_lib_device_status(_stream(stream), 1 if reset else 0))

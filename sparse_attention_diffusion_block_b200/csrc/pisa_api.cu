@@ -1,0 +1,364 @@
+// C ABI of the PISA library: argument validation, workspace carve-up and the
+// launch sequence stats -> Hbar -> covariance norm -> routing -> fused forward.
+// Every entry point validates on the host before any launch.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+
+#include "common.cuh"
+#include "fused_simt.cuh"
+#include "select.cuh"
+#include "stats_simt.cuh"
+
+namespace pisa {
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Shape {
+  int batch, heads, L, d, block;
+  int BH() const { return batch * heads; }
+  int nb() const { return (L + block - 1) / block; }
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+pisa_status check_shape(const Shape& s) {
+  if (s.batch < 1 || s.heads < 1 || s.L < 1 || s.d < 1 || s.block < 1) return PISA_ERR_INVALID_ARG;
+  if ((long long)s.batch * s.heads > 65535) return PISA_ERR_UNSUPPORTED;
+  if (s.d != 64 && s.d != 128) return PISA_ERR_UNSUPPORTED;
+  if (s.block != 64 && s.block != 128) return PISA_ERR_UNSUPPORTED;
+  if ((long long)s.L * s.d * s.batch * s.heads > (1LL << 40)) return PISA_ERR_UNSUPPORTED;
+  return PISA_OK;
+}
+
+template <typename... P>
+bool all_ok(P... p) {
+  const void* ptrs[] = {static_cast<const void*>(p)...};
+  for (const void* x : ptrs)
+    if (x == nullptr || !aligned16(x)) return false;
+  return true;
+}
+
+// Blocks per stats CTA: enough CTAs to fill the GPU a few times over while
+// keeping the partial-sum traffic (one d x d tile per CTA) small.
+int stats_chunk(const Shape& s) {
+  const long long target = 4LL * 148;
+  long long J = ((long long)s.BH() * s.nb()) / target;
+  if (J < 1) J = 1;
+  if (J > s.nb()) J = s.nb();
+  return (int)J;
+}
+int stats_chunks(const Shape& s) {
+  const int J = stats_chunk(s);
+  return (s.nb() + J - 1) / J;
+}
+
+size_t stats_ws(const Shape& s) {
+  return align_up((size_t)s.BH() * stats_chunks(s) * s.d * s.d * sizeof(float));
+}
+
+size_t fused_ws(const Shape&) { return 0; }
+
+struct Carve {
+  float *qbar, *kbar, *vsum, *hbar, *M;
+  int32_t* sel;
+  void* stats;
+  void* fused;
+  size_t total;
+};
+
+Carve carve(const Shape& s, int k, char* base) {
+  Carve c{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* p = base ? base + off : nullptr;
+    off += align_up(bytes);
+    return p;
+  };
+  const size_t stat = (size_t)s.BH() * s.nb() * s.d * sizeof(float);
+  c.qbar = reinterpret_cast<float*>(take(stat));
+  c.kbar = reinterpret_cast<float*>(take(stat));
+  c.vsum = reinterpret_cast<float*>(take(stat));
+  c.hbar = reinterpret_cast<float*>(take((size_t)s.BH() * s.d * s.d * sizeof(float)));
+  c.M = reinterpret_cast<float*>(take((size_t)s.BH() * s.nb() * sizeof(float)));
+  c.sel = reinterpret_cast<int32_t*>(take((size_t)s.BH() * s.nb() * k * sizeof(int32_t)));
+  c.stats = take(stats_ws(s));
+  c.fused = take(fused_ws(s) ? fused_ws(s) : 16);
+  c.total = off;
+  return c;
+}
+
+pisa_status last_launch() {
+  return cudaGetLastError() == cudaSuccess ? PISA_OK : PISA_ERR_CUDA;
+}
+
+template <typename F>
+bool set_smem(F* kernel, size_t bytes) {
+  if (bytes <= 48 * 1024) return true;
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) ==
+         cudaSuccess;
+}
+
+// ------------------------------------------------------------------ stages
+
+template <typename T, int D>
+pisa_status run_stats(const T* q, const T* k, const T* v, const Shape& s, float* qbar, float* kbar,
+                      float* vsum, float* hbar, float* partial, cudaStream_t st) {
+  const int J = stats_chunk(s), nc = stats_chunks(s);
+  const size_t smem = (2 * (size_t)s.block * (D + 4) + 2 * D + 256) * sizeof(float);
+  if (!set_smem(stats_simt_kernel<T, D>, smem)) return PISA_ERR_CUDA;
+  stats_simt_kernel<T, D><<<dim3(nc, s.BH()), 256, smem, st>>>(q, k, v, s.L, s.block, s.nb(), J, qbar,
+                                                                kbar, vsum, partial);
+  if (last_launch() != PISA_OK) return PISA_ERR_CUDA;
+  hbar_reduce_kernel<D><<<dim3((D * D + 255) / 256, s.BH()), 256, 0, st>>>(partial, nc, s.nb(), hbar);
+  return last_launch();
+}
+
+template <typename T, int D, bool WRITE_H>
+pisa_status run_block_h(const T* k, const T* v, const Shape& s, const float* kbar, const float* vsum,
+                        const float* hbar, float* out, cudaStream_t st) {
+  const size_t smem = (2 * (size_t)s.block * (D + 4) + 8) * sizeof(float);
+  if (!set_smem(block_h_simt_kernel<T, D, WRITE_H>, smem)) return PISA_ERR_CUDA;
+  block_h_simt_kernel<T, D, WRITE_H><<<dim3(s.nb(), s.BH()), 256, smem, st>>>(
+      k, v, s.L, s.block, s.nb(), kbar, vsum, hbar, out);
+  return last_launch();
+}
+
+int select_rows(int nb) {
+  const long long budget = 150 * 1024;
+  long long R = budget / (4LL * nb);
+  if (R > 32) R = 32;
+  return (int)R;
+}
+
+template <int D>
+pisa_status run_select(const float* qbar, const float* kbar, const float* M, const Shape& s, int k,
+                       int32_t* sel, cudaStream_t st) {
+  const int nb = s.nb();
+  const int R = select_rows(nb);
+  if (R < 1) return PISA_ERR_UNSUPPORTED;
+  const size_t smem = ((size_t)R * D + 32 * (D + 4) + R + 64 + (size_t)R * nb) * sizeof(float);
+  if (!set_smem(select_kernel<D>, smem)) return PISA_ERR_CUDA;
+  const float scale = 1.0f / sqrtf((float)D);
+  select_kernel<D><<<dim3((nb + R - 1) / R, s.BH()), 256, smem, st>>>(qbar, kbar, M, s.L, s.block, nb,
+                                                                      k, R, scale, sel);
+  return last_launch();
+}
+
+template <typename T, int D>
+pisa_status run_fused(const T* q, const T* k, const T* v, T* out, const Shape& s, const float* kbar,
+                      const float* vsum, const float* hbar, const int32_t* sel, int kk,
+                      cudaStream_t st) {
+  constexpr int TPR = 4, CH = 16, DS = D / TPR, RS = TPR * (DS + 4);
+  const int nb = s.nb();
+  const size_t smem = (2 * (size_t)CH * RS + (size_t)D * D + CH + (nb + 31) / 32) * sizeof(float);
+  if (!set_smem(fused_simt_kernel<T, D, TPR, CH>, smem)) return PISA_ERR_CUDA;
+  const float scale = 1.0f / sqrtf((float)D);
+  fused_simt_kernel<T, D, TPR, CH><<<dim3(nb, s.BH()), s.block * TPR, smem, st>>>(
+      q, k, v, out, s.L, s.block, nb, kk, kbar, vsum, hbar, sel, scale);
+  return last_launch();
+}
+
+// dtype / d dispatch helpers
+template <template <typename, int> class Op, typename... A>
+pisa_status dispatch(pisa_dtype dt, int d, A&&... a) {
+  if (dt == PISA_BF16) {
+    if (d == 128) return Op<__nv_bfloat16, 128>::run(a...);
+    if (d == 64) return Op<__nv_bfloat16, 64>::run(a...);
+  } else if (dt == PISA_FP32) {
+    if (d == 128) return Op<float, 128>::run(a...);
+    if (d == 64) return Op<float, 64>::run(a...);
+  }
+  return PISA_ERR_UNSUPPORTED;
+}
+
+template <typename T, int D>
+struct StatsOp {
+  static pisa_status run(const void* q, const void* k, const void* v, const Shape& s, float* qbar,
+                         float* kbar, float* vsum, float* hbar, float* partial, cudaStream_t st) {
+    return run_stats<T, D>((const T*)q, (const T*)k, (const T*)v, s, qbar, kbar, vsum, hbar, partial, st);
+  }
+};
+
+template <typename T, int D>
+struct CovNormOp {
+  static pisa_status run(const void* k, const void* v, const Shape& s, const float* kbar,
+                         const float* vsum, const float* hbar, float* M, cudaStream_t st) {
+    return run_block_h<T, D, false>((const T*)k, (const T*)v, s, kbar, vsum, hbar, M, st);
+  }
+};
+
+template <typename T, int D>
+struct FirstOrderOp {
+  static pisa_status run(const void* k, const void* v, const Shape& s, const float* kbar,
+                         const float* vsum, float* H, cudaStream_t st) {
+    return run_block_h<T, D, true>((const T*)k, (const T*)v, s, kbar, vsum, nullptr, H, st);
+  }
+};
+
+template <typename T, int D>
+struct FusedOp {
+  static pisa_status run(const void* q, const void* k, const void* v, void* out, const Shape& s,
+                         const float* kbar, const float* vsum, const float* hbar, const int32_t* sel,
+                         int kk, void* ws, cudaStream_t st) {
+    (void)ws;
+    return run_fused<T, D>((const T*)q, (const T*)k, (const T*)v, (T*)out, s, kbar, vsum, hbar, sel, kk,
+                           st);
+  }
+};
+
+bool valid_dtype(pisa_dtype dt) { return dt == PISA_BF16 || dt == PISA_FP32; }
+
+}  // namespace
+}  // namespace pisa
+
+using namespace pisa;
+
+extern "C" {
+
+const char* pisa_status_string(pisa_status status) {
+  switch (status) {
+    case PISA_OK: return "ok";
+    case PISA_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, bad size)";
+    case PISA_ERR_UNSUPPORTED: return "unsupported shape (d and block must be 64 or 128)";
+    case PISA_ERR_WORKSPACE: return "workspace missing or too small";
+    case PISA_ERR_CUDA: return "CUDA runtime error";
+    case PISA_ERR_TIMEOUT: return "a bounded device wait timed out";
+    case PISA_ERR_DEVICE_CHECK: return "a device-side index check failed";
+  }
+  return "unknown status";
+}
+
+int pisa_keep_count(int L, int block, float keep_ratio) {
+  if (L < 1 || block < 1 || !std::isfinite(keep_ratio) || keep_ratio <= 0.f) return -1;
+  const long long nb = ((long long)L + block - 1) / block;
+  long long k = (long long)std::ceil((double)keep_ratio * (double)nb - 1e-9);
+  if (k < 1) k = 1;
+  if (k > nb) k = nb;
+  return (int)k;
+}
+
+size_t pisa_stats_workspace_size(int batch, int heads, int L, int d, int block) {
+  const Shape s{batch, heads, L, d, block};
+  if (check_shape(s) != PISA_OK) return 0;
+  return stats_ws(s);
+}
+
+size_t pisa_fused_workspace_size(int batch, int heads, int L, int d, int block) {
+  const Shape s{batch, heads, L, d, block};
+  if (check_shape(s) != PISA_OK) return 0;
+  return fused_ws(s);
+}
+
+size_t pisa_workspace_size(int batch, int heads, int L, int d, int block, int k) {
+  const Shape s{batch, heads, L, d, block};
+  if (check_shape(s) != PISA_OK || k < 1 || k > s.nb()) return 0;
+  return carve(s, k, nullptr).total;
+}
+
+pisa_status pisa_block_stats(const void* q, const void* k, const void* v, pisa_dtype dtype, int batch,
+                             int heads, int L, int d, int block, float* qbar, float* kbar, float* vsum,
+                             float* hbar, void* workspace, size_t workspace_bytes, void* stream) {
+  const Shape s{batch, heads, L, d, block};
+  if (pisa_status e = check_shape(s)) return e;
+  if (!valid_dtype(dtype)) return PISA_ERR_INVALID_ARG;
+  if (!all_ok(q, k, v, qbar, kbar, vsum, hbar)) return PISA_ERR_INVALID_ARG;
+  if (workspace == nullptr || workspace_bytes < stats_ws(s)) return PISA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return PISA_ERR_INVALID_ARG;
+  return dispatch<StatsOp>(dtype, d, q, k, v, s, qbar, kbar, vsum, hbar, (float*)workspace,
+                           (cudaStream_t)stream);
+}
+
+pisa_status pisa_cov_norm(const void* k, const void* v, pisa_dtype dtype, int batch, int heads, int L,
+                          int d, int block, const float* kbar, const float* vsum, const float* hbar,
+                          float* M, void* stream) {
+  const Shape s{batch, heads, L, d, block};
+  if (pisa_status e = check_shape(s)) return e;
+  if (!valid_dtype(dtype)) return PISA_ERR_INVALID_ARG;
+  if (!all_ok(k, v, kbar, vsum, hbar, M)) return PISA_ERR_INVALID_ARG;
+  return dispatch<CovNormOp>(dtype, d, k, v, s, kbar, vsum, hbar, M, (cudaStream_t)stream);
+}
+
+pisa_status pisa_block_first_order(const void* k, const void* v, pisa_dtype dtype, int batch, int heads,
+                                   int L, int d, int block, const float* kbar, const float* vsum,
+                                   float* H, void* stream) {
+  const Shape s{batch, heads, L, d, block};
+  if (pisa_status e = check_shape(s)) return e;
+  if (!valid_dtype(dtype)) return PISA_ERR_INVALID_ARG;
+  if (!all_ok(k, v, kbar, vsum, H)) return PISA_ERR_INVALID_ARG;
+  return dispatch<FirstOrderOp>(dtype, d, k, v, s, kbar, vsum, H, (cudaStream_t)stream);
+}
+
+pisa_status pisa_select(const float* qbar, const float* kbar, const float* M, int batch, int heads, int L,
+                        int d, int block, int k, int32_t* sel, void* stream) {
+  const Shape s{batch, heads, L, d, block};
+  if (pisa_status e = check_shape(s)) return e;
+  if (k < 1 || k > s.nb()) return PISA_ERR_INVALID_ARG;
+  if (!all_ok(qbar, kbar, M) || sel == nullptr || (reinterpret_cast<uintptr_t>(sel) & 3u))
+    return PISA_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  return d == 128 ? run_select<128>(qbar, kbar, M, s, k, sel, st)
+                  : run_select<64>(qbar, kbar, M, s, k, sel, st);
+}
+
+pisa_status pisa_attn_fwd_with_sel(const void* q, const void* k, const void* v, void* out, pisa_dtype dtype,
+                                   int batch, int heads, int L, int d, int block, const float* kbar,
+                                   const float* vsum, const float* hbar, const int32_t* sel, int k_sel,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  const Shape s{batch, heads, L, d, block};
+  if (pisa_status e = check_shape(s)) return e;
+  if (!valid_dtype(dtype)) return PISA_ERR_INVALID_ARG;
+  if (k_sel < 1 || k_sel > s.nb()) return PISA_ERR_INVALID_ARG;
+  if (!all_ok(q, k, v, out, kbar, vsum, hbar) || sel == nullptr) return PISA_ERR_INVALID_ARG;
+  if (fused_ws(s) && (workspace == nullptr || workspace_bytes < fused_ws(s))) return PISA_ERR_WORKSPACE;
+  return dispatch<FusedOp>(dtype, d, q, k, v, out, s, kbar, vsum, hbar, sel, k_sel, workspace,
+                           (cudaStream_t)stream);
+}
+
+pisa_status pisa_attn_fwd(const void* q, const void* k, const void* v, void* out, pisa_dtype dtype, int batch,
+                          int heads, int L, int d, int block, float keep_ratio, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  const Shape s{batch, heads, L, d, block};
+  if (pisa_status e = check_shape(s)) return e;
+  if (!valid_dtype(dtype)) return PISA_ERR_INVALID_ARG;
+  const int kk = pisa_keep_count(L, block, keep_ratio);
+  if (kk < 1) return PISA_ERR_INVALID_ARG;
+  if (!all_ok(q, k, v, out)) return PISA_ERR_INVALID_ARG;
+  const Carve need = carve(s, kk, nullptr);
+  if (workspace == nullptr || workspace_bytes < need.total) return PISA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return PISA_ERR_INVALID_ARG;
+  const Carve c = carve(s, kk, static_cast<char*>(workspace));
+  cudaStream_t st = (cudaStream_t)stream;
+  pisa_status e = dispatch<StatsOp>(dtype, d, q, k, v, s, c.qbar, c.kbar, c.vsum, c.hbar, (float*)c.stats, st);
+  if (e) return e;
+  e = dispatch<CovNormOp>(dtype, d, k, v, s, (const float*)c.kbar, (const float*)c.vsum,
+                          (const float*)c.hbar, c.M, st);
+  if (e) return e;
+  e = d == 128 ? run_select<128>(c.qbar, c.kbar, c.M, s, kk, c.sel, st)
+               : run_select<64>(c.qbar, c.kbar, c.M, s, kk, c.sel, st);
+  if (e) return e;
+  return dispatch<FusedOp>(dtype, d, q, k, v, out, s, (const float*)c.kbar, (const float*)c.vsum,
+                           (const float*)c.hbar, (const int32_t*)c.sel, kk, c.fused, st);
+}
+
+pisa_status pisa_device_status(void* stream, int reset) {
+  cudaStream_t st = (cudaStream_t)stream;
+  int word = 0;
+  if (cudaMemcpyFromSymbolAsync(&word, g_error_word, sizeof(int), 0, cudaMemcpyDeviceToHost, st) !=
+      cudaSuccess)
+    return PISA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return PISA_ERR_CUDA;
+  if (reset && word != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbolAsync(g_error_word, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+      return PISA_ERR_CUDA;
+  }
+  if (word == 0) return PISA_OK;
+  return (pisa_status)word;
+}
+
+}  // extern "C"

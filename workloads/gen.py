@@ -230,7 +230,8 @@ def generate(cfg: Config, heads: Optional[Iterable[int]] = None,
     k = np.empty(shape, dtype=np.float32)
     v = np.empty(shape, dtype=np.float32)
     if workers is None:
-        workers = min(len(bhs), os.cpu_count() or 1, 16)
+        big = len(bhs) * cfg.L * cfg.d >= 4_000_000
+        workers = min(len(bhs), os.cpu_count() or 1, 16) if big else 1
     if workers <= 1 or len(bhs) <= 1:
         for n, bh in enumerate(bhs):
             q[n], k[n], v[n] = generate_head(cfg, bh, redraws.get(bh))
