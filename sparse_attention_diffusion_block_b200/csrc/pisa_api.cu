@@ -4,9 +4,11 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <type_traits>
 
 #include "common.cuh"
 #include "fused_simt.cuh"
+#include "fused_sm100.cuh"
 #include "select.cuh"
 #include "stats_simt.cuh"
 
@@ -59,7 +61,13 @@ size_t stats_ws(const Shape& s) {
   return align_up((size_t)s.BH() * stats_chunks(s) * s.d * s.d * sizeof(float));
 }
 
-size_t fused_ws(const Shape&) { return 0; }
+// bf16 hi/lo operands of the tensor-core fused kernel: centroid keys and
+// value sums [BH][2*nbp][d], Hbar transposed [BH][2*d][d].
+int padded_blocks(const Shape& s) { return (s.nb() + 127) / 128 * 128; }
+size_t fused_ws(const Shape& s) {
+  const size_t cent = align_up((size_t)s.BH() * 2 * padded_blocks(s) * s.d * 2);
+  return 2 * cent + align_up((size_t)s.BH() * 2 * s.d * s.d * 2);
+}
 
 struct Carve {
   float *qbar, *kbar, *vsum, *hbar, *M;
@@ -85,7 +93,7 @@ Carve carve(const Shape& s, int k, char* base) {
   c.M = reinterpret_cast<float*>(take((size_t)s.BH() * s.nb() * sizeof(float)));
   c.sel = reinterpret_cast<int32_t*>(take((size_t)s.BH() * s.nb() * k * sizeof(int32_t)));
   c.stats = take(stats_ws(s));
-  c.fused = take(fused_ws(s) ? fused_ws(s) : 16);
+  c.fused = take(fused_ws(s));
   c.total = off;
   return c;
 }
@@ -161,6 +169,72 @@ pisa_status run_fused(const T* q, const T* k, const T* v, T* out, const Shape& s
   return last_launch();
 }
 
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_fn() {
+  static EncodeTiled fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(p);
+  }
+  return fn;
+}
+
+// 3-D bf16 map over [outer][rows][inner] with 64-element (128-byte) swizzled
+// boxes of `box_rows` rows; reads outside [0, rows) return zeros.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer, uint32_t box_rows) {
+  EncodeTiled fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {inner, rows, outer};
+  const cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
+  const cuuint32_t box[3] = {64, box_rows, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int KB>
+pisa_status run_fused_sm100(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                            __nv_bfloat16* out, const Shape& s, const float* kbar, const float* vsum,
+                            const float* hbar, const int32_t* sel, int kk, void* ws, cudaStream_t st) {
+  const int nb = s.nb(), nbp = padded_blocks(s), BH = s.BH();
+  char* w = static_cast<char*>(ws);
+  const size_t cent = align_up((size_t)BH * 2 * nbp * D * 2);
+  __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(w);
+  __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(w + cent);
+  __nv_bfloat16* ht = reinterpret_cast<__nv_bfloat16*>(w + 2 * cent);
+  const int elems = nbp * D > D * D ? nbp * D : D * D;
+  prep_fused_operands_kernel<D><<<dim3((elems + 255) / 256, BH), 256, 0, st>>>(kbar, vsum, hbar, nb, nbp, kc, vc, ht);
+  if (last_launch() != PISA_OK) return PISA_ERR_CUDA;
+  CUtensorMap mQ, mK, mV, mKc, mVc, mH;
+  if (!make_map(&mQ, q, D, s.L, BH, 128) || !make_map(&mK, k, D, s.L, BH, KB) || !make_map(&mV, v, D, s.L, BH, KB) ||
+      !make_map(&mKc, kc, D, 2 * nbp, BH, 128) || !make_map(&mVc, vc, D, 2 * nbp, BH, 128) ||
+      !make_map(&mH, ht, D, 2 * D, BH, D))
+    return PISA_ERR_CUDA;
+  constexpr int G = 128 / KB;
+  const size_t smem = FusedLayout<D>::bytes(G, kk, nbp);
+  if (smem > 227 * 1024) return PISA_ERR_UNSUPPORTED;
+  if (!set_smem(fused_sm100_kernel<D, KB>, smem)) return PISA_ERR_CUDA;
+  FusedArgs fa;
+  fa.sel = sel;
+  fa.out = out;
+  fa.kk = kk;
+  fa.L = s.L;
+  fa.nb = nb;
+  fa.nbp = nbp;
+  fa.block = s.block;
+  fa.scale = 1.0f / sqrtf((float)D);
+  fa.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
+  fused_sm100_kernel<D, KB><<<dim3((s.L + 127) / 128, BH), kFusedThreads, smem, st>>>(mQ, mK, mV, mKc, mVc, mH, fa);
+  return last_launch();
+}
+
 // dtype / d dispatch helpers
 template <template <typename, int> class Op, typename... A>
 pisa_status dispatch(pisa_dtype dt, int d, A&&... a) {
@@ -198,14 +272,24 @@ struct FirstOrderOp {
   }
 };
 
+// fp32 inputs: CUDA-core fused kernel (tf32 MMAs cannot hold the fp32
+// tolerance).  bf16 inputs: the tcgen05 tensor-core kernel.
 template <typename T, int D>
 struct FusedOp {
   static pisa_status run(const void* q, const void* k, const void* v, void* out, const Shape& s,
                          const float* kbar, const float* vsum, const float* hbar, const int32_t* sel,
                          int kk, void* ws, cudaStream_t st) {
-    (void)ws;
-    return run_fused<T, D>((const T*)q, (const T*)k, (const T*)v, (T*)out, s, kbar, vsum, hbar, sel, kk,
-                           st);
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+      using B16 = __nv_bfloat16;
+      if (s.block == 128)
+        return run_fused_sm100<D, 128>((const B16*)q, (const B16*)k, (const B16*)v, (B16*)out, s, kbar, vsum,
+                                       hbar, sel, kk, ws, st);
+      return run_fused_sm100<D, 64>((const B16*)q, (const B16*)k, (const B16*)v, (B16*)out, s, kbar, vsum, hbar,
+                                    sel, kk, ws, st);
+    } else {
+      (void)ws;
+      return run_fused<T, D>((const T*)q, (const T*)k, (const T*)v, (T*)out, s, kbar, vsum, hbar, sel, kk, st);
+    }
   }
 };
 
@@ -312,7 +396,8 @@ pisa_status pisa_attn_fwd_with_sel(const void* q, const void* k, const void* v, 
   if (!valid_dtype(dtype)) return PISA_ERR_INVALID_ARG;
   if (k_sel < 1 || k_sel > s.nb()) return PISA_ERR_INVALID_ARG;
   if (!all_ok(q, k, v, out, kbar, vsum, hbar) || sel == nullptr) return PISA_ERR_INVALID_ARG;
-  if (fused_ws(s) && (workspace == nullptr || workspace_bytes < fused_ws(s))) return PISA_ERR_WORKSPACE;
+  if (dtype == PISA_BF16 && (workspace == nullptr || workspace_bytes < fused_ws(s))) return PISA_ERR_WORKSPACE;
+  if (workspace != nullptr && !aligned16(workspace)) return PISA_ERR_INVALID_ARG;
   return dispatch<FusedOp>(dtype, d, q, k, v, out, s, kbar, vsum, hbar, sel, k_sel, workspace,
                            (cudaStream_t)stream);
 }
