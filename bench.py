@@ -270,10 +270,15 @@ def main():
                     help="seconds of oracle time for the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="run only the first N heads of the workload (profiling captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     cfg = workload_config(args.workload)
+    if args.heads is not None:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, heads=min(args.heads, cfg.heads))
 
     if args.impl == "reference":
         import oracle  # reference arm: the oracle as it stands
@@ -438,7 +443,7 @@ def main():
             "stages": stages,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": K * pisa.LAUNCHES["attn_fwd"],
+            "gpu_launches": K * pisa.launches("attn_fwd", tdt),
             "clocks": clocks.summary(),
         }
         print(json.dumps(line), flush=True)

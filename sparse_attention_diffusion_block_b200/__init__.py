@@ -217,9 +217,12 @@ def attn_fwd(q, k, v, block, keep_ratio, out=None, workspace=None, stream=None):
     return out
 
 
-# Kernels each entry point launches (for launch accounting in the bench).
-LAUNCHES = {"block_stats": 2, "cov_norm": 1, "select": 1, "attn_fwd_with_sel": 1}
-LAUNCHES["attn_fwd"] = sum(LAUNCHES.values())
+def launches(entry: str, dtype: torch.dtype = torch.bfloat16) -> int:
+    """Number of kernels an entry point launches (launch accounting)."""
+    fused = 2 if dtype == torch.bfloat16 else 1  # bf16: operand prep + tensor-core kernel
+    table = {"block_stats": 2, "cov_norm": 1, "select": 1, "attn_fwd_with_sel": fused}
+    table["attn_fwd"] = sum(table.values())
+    return table[entry]
 
 
 def device_status(stream=None, reset: bool = True) -> int:

@@ -11,6 +11,7 @@
 #include "fused_sm100.cuh"
 #include "select.cuh"
 #include "stats_simt.cuh"
+#include "stats_sm100.cuh"
 
 namespace pisa {
 namespace {
@@ -43,10 +44,10 @@ bool all_ok(P... p) {
   return true;
 }
 
-// Blocks per stats CTA: enough CTAs to fill the GPU a few times over while
-// keeping the partial-sum traffic (one d x d tile per CTA) small.
+// Blocks per stats CTA: enough CTAs to fill the 148 SMs several times over
+// while keeping the partial-sum traffic (one d x d tile per CTA) small.
 int stats_chunk(const Shape& s) {
-  const long long target = 4LL * 148;
+  const long long target = 6LL * 148;
   long long J = ((long long)s.BH() * s.nb()) / target;
   if (J < 1) J = 1;
   if (J > s.nb()) J = s.nb();
@@ -111,10 +112,33 @@ bool set_smem(F* kernel, size_t bytes) {
 
 // ------------------------------------------------------------------ stages
 
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer, uint32_t box_rows);
+
 template <typename T, int D>
 pisa_status run_stats(const T* q, const T* k, const T* v, const Shape& s, float* qbar, float* kbar,
                       float* vsum, float* hbar, float* partial, cudaStream_t st) {
   const int J = stats_chunk(s), nc = stats_chunks(s);
+  if constexpr (std::is_same<T, __nv_bfloat16>::value && D == 128) {
+    CUtensorMap mQ, mK, mV;
+    const uint32_t box = (uint32_t)s.block;
+    if (!make_map(&mQ, q, D, s.L, s.BH(), box) || !make_map(&mK, k, D, s.L, s.BH(), box) ||
+        !make_map(&mV, v, D, s.L, s.BH(), box))
+      return PISA_ERR_CUDA;
+    if (s.block == 128) {
+      const size_t smem = StatsLayout<128>::bytes();
+      if (!set_smem(stats_sm100_kernel<128>, smem)) return PISA_ERR_CUDA;
+      stats_sm100_kernel<128><<<dim3(nc, s.BH()), kStatsThreads, smem, st>>>(mQ, mK, mV, s.L, s.nb(), J, qbar,
+                                                                              kbar, vsum, partial);
+    } else {
+      const size_t smem = StatsLayout<64>::bytes();
+      if (!set_smem(stats_sm100_kernel<64>, smem)) return PISA_ERR_CUDA;
+      stats_sm100_kernel<64><<<dim3(nc, s.BH()), kStatsThreads, smem, st>>>(mQ, mK, mV, s.L, s.nb(), J, qbar,
+                                                                            kbar, vsum, partial);
+    }
+    if (last_launch() != PISA_OK) return PISA_ERR_CUDA;
+    hbar_reduce_kernel<D><<<dim3((D * D + 255) / 256, s.BH()), 256, 0, st>>>(partial, nc, s.nb(), hbar);
+    return last_launch();
+  }
   const size_t smem = (2 * (size_t)s.block * (D + 4) + 2 * D + 256) * sizeof(float);
   if (!set_smem(stats_simt_kernel<T, D>, smem)) return PISA_ERR_CUDA;
   stats_simt_kernel<T, D><<<dim3(nc, s.BH()), 256, smem, st>>>(q, k, v, s.L, s.block, s.nb(), J, qbar,
@@ -124,9 +148,34 @@ pisa_status run_stats(const T* q, const T* k, const T* v, const Shape& s, float*
   return last_launch();
 }
 
+int cov_chunk(const Shape& s) {
+  long long J = ((long long)s.BH() * s.nb() + 8LL * 148 - 1) / (8LL * 148);
+  if (J < 1) J = 1;
+  if (J > s.nb()) J = s.nb();
+  return (int)J;
+}
+
 template <typename T, int D, bool WRITE_H>
 pisa_status run_block_h(const T* k, const T* v, const Shape& s, const float* kbar, const float* vsum,
                         const float* hbar, float* out, cudaStream_t st) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value && D == 128 && !WRITE_H) {
+    CUtensorMap mK, mV;
+    const uint32_t box = (uint32_t)s.block;
+    if (!make_map(&mK, k, D, s.L, s.BH(), box) || !make_map(&mV, v, D, s.L, s.BH(), box)) return PISA_ERR_CUDA;
+    const int J = cov_chunk(s), nc = (s.nb() + J - 1) / J;
+    if (s.block == 128) {
+      const size_t smem = StatsLayout<128>::bytes();
+      if (!set_smem(cov_norm_sm100_kernel<128>, smem)) return PISA_ERR_CUDA;
+      cov_norm_sm100_kernel<128><<<dim3(nc, s.BH()), kStatsThreads, smem, st>>>(mK, mV, s.L, s.nb(), J, kbar, vsum,
+                                                                                hbar, out);
+    } else {
+      const size_t smem = StatsLayout<64>::bytes();
+      if (!set_smem(cov_norm_sm100_kernel<64>, smem)) return PISA_ERR_CUDA;
+      cov_norm_sm100_kernel<64><<<dim3(nc, s.BH()), kStatsThreads, smem, st>>>(mK, mV, s.L, s.nb(), J, kbar, vsum,
+                                                                               hbar, out);
+    }
+    return last_launch();
+  }
   const size_t smem = (2 * (size_t)s.block * (D + 4) + 8) * sizeof(float);
   if (!set_smem(block_h_simt_kernel<T, D, WRITE_H>, smem)) return PISA_ERR_CUDA;
   block_h_simt_kernel<T, D, WRITE_H><<<dim3(s.nb(), s.BH()), 256, smem, st>>>(

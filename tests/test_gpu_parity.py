@@ -77,7 +77,10 @@ def test_small_shapes_every_stage(lib, cfg):
             assert_stat_close(g["vsum"][b, h], r["vsum"], 1e-5, tag + " vsum")
             assert_stat_close(g["H"][b, h], r["H"], 1e-5, tag + " H")
             assert_stat_close(g["hbar"][b, h], r["Hbar"], 1e-4, tag + " Hbar")
-            assert_stat_close(g["M"][b, h], r["M"], 1e-5, tag + " M")
+            # M_j is a norm of H_j - Hbar: rounding in it scales with ||H_j||_F,
+            # not with M_j (which is exactly 0 when nb = 1)
+            h_scale = np.sqrt((r["H"] ** 2).sum(axis=(1, 2))).max()
+            assert np.abs(g["M"][b, h] - r["M"]).max() <= 1e-5 * max(h_scale, 1e-30), tag + " M"
             np.testing.assert_array_equal(g["sel"][b, h], r["sel"], err_msg=tag + " S_i")
             assert_output_close(g["out"][b, h], r["out"], cfg.dtype, tag)
 
