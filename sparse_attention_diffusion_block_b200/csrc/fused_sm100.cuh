@@ -4,25 +4,33 @@
 // equation, alpha_{t,j} = exp(q_t kbar_j^T)) and hardware implementation
 // (phase 1: exact attention over the selected blocks; phase 2: zeroth-order
 // scan over the unselected blocks' aggregated vectors; phase 3: the global
-// first-order correction), all folded into ONE online softmax.
+// first-order correction), all folded into ONE online softmax per row.
 //
-// One CTA per 128-row query tile of one (batch, head).  Warp roles:
-//   warps 0-3  softmax: one thread per query row (= TMEM lane).  Reads S from
-//              TMEM, keeps the running max m, l = D e^{-m}, beta e^{-m},
-//              writes P (bf16) back over S for the PV MMA, rescales O in TMEM
-//              when the max grows by more than 2^8 (lazy rescale; exact because
-//              N and D carry the same factor), epilogue.
-//   warp 4     TMA producer: Q once, then a ring of 128-row operand tiles.
-//   warp 5     MMA issuer (one thread): S = Q K^T into a double-buffered TMEM
-//              accumulator, O += P V with P read from TMEM.
-// Tile sequence: the exact KV blocks of the tile's query block(s) (their
-// union when a tile spans two 64-token blocks, with a per-row-group mask),
-// then the centroid tiles (128 key centroids each; k and v are fp32 stats
-// fed as bf16 hi + lo pairs, two MMAs each); the first-order term q_t Hbar
-// (Hbar as hi + lo) is one more MMA into its own TMEM columns.
+// Persistent CTAs, one per SM, walk "pairs" of consecutive 128-row query
+// tiles (A, B) of one (batch, head), head-major so that the ~150 pairs in
+// flight share one or two heads' K/V in L2.  Warp roles (384 threads; the
+// softmax warpgroups raise their register limit to 200 with setmaxnreg, the
+// third warpgroup drops to 104):
+//   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: one thread per
+//              query row (= TMEM lane).  Reads S, keeps the running max m, l =
+//              D e^{-m} and beta e^{-m}, writes P (bf16) over S for the PV MMA,
+//              rescales O in TMEM when m grows by more than 8 (log2 units;
+//              exact since N and D carry the same factor), epilogue
+//              o = (O + s beta q Hbar) / l.
+//   warp 8     producer: builds each pair's work list in shared memory, then
+//              streams Q tiles and a ring of 128-row operand tiles with TMA.
+//   warp 9     MMA issuer (one thread): S = Q K^T and O += P V (P from TMEM),
+//              ping-ponging the two tiles so that one tile's softmax overlaps
+//              the other tile's MMAs.
+// Work list of a pair: the exact KV blocks of each tile (for 64-token blocks a
+// 128-row tile spans two query blocks: the union, with per-row-group bits),
+// blocks selected by both tiles first and in the same order, so those K/V
+// tiles are loaded once and feed both; then the centroid tiles (128 key
+// centroids each, shared by both tiles, masked per tile); fp32 statistics
+// enter as bf16 hi + lo MMA pairs.  q_t Hbar (Hbar as hi + lo) runs last into
+// the tile's S columns.
 //
-// TMEM columns: [0,128) S buffer 0, [128,256) S buffer 1, [256,256+D) O,
-// [256+D, 256+2D) q Hbar.
+// TMEM columns: [0,128) S_A, [128,256) S_B, [256,256+D) O_A, [256+D,256+2D) O_B.
 #pragma once
 
 #include "sm100.cuh"
@@ -33,11 +41,13 @@ struct FusedArgs {
   const int32_t* sel;
   __nv_bfloat16* out;
   int kk, L, nb, nbp, block;
+  int n_qtiles;  // 128-row query tiles per (batch, head)
+  int n_pairs;   // BH * ceil(n_qtiles / 2)
   float scale;       // 1/sqrt(d)
   float scale_log2;  // log2(e)/sqrt(d)
 };
 
-constexpr int kFusedThreads = 192;
+constexpr int kFusedThreads = 384;  // 3 warpgroups: softmax A, softmax B, producer/MMA
 constexpr int kFusedStages = 4;
 
 template <int D>
@@ -46,13 +56,42 @@ struct FusedLayout {
   static constexpr uint32_t kSlot = 128u * D * 2u;  // one operand tile
   static constexpr uint32_t kQ = QT * D * 2u;
   static constexpr uint32_t kRing = kFusedStages * kSlot;
-  static constexpr uint32_t kBars = (2 * kFusedStages + 8) * 8u;
-  static constexpr uint32_t kFixed = kQ + kRing + kBars + 16;
-  // + list (G*kk ints) + masks (G * nbp/32 words), + 1024 alignment slack
+  static constexpr int kNumBars = 2 * kFusedStages + 18;
+  static constexpr uint32_t kBars = kNumBars * 8u;
+  // one work-list slot: header[8] + entries A/B [G*kk each] + masks A/B [G*words each]
+  __host__ __device__ static size_t list_ints(int G, int kk, int words) { return 8 + 2 * (size_t)G * kk + 2 * (size_t)G * words; }
   static size_t bytes(int G, int kk, int nbp) {
-    return 1024 + kFixed + sizeof(int) * (size_t)G * kk + sizeof(uint32_t) * (size_t)G * (nbp / 32);
+    return 1024 + 2 * kQ + kRing + kBars + 16 + 2 * 4 * list_ints(G, kk, nbp / 32);
   }
 };
+
+// Step structure of a pair, shared by the producer and the MMA issuer so that
+// both walk the ring items in exactly the same order.
+struct PairPlan {
+  int nA, nB, nC, existsB, ncent;
+  __device__ int U() const { return nA > nB ? nA : nB; }
+  __device__ int T() const { return U() + ncent; }
+  __device__ bool activeA(int u) const { return u < nA || u >= U(); }
+  __device__ bool activeB(int u) const { return existsB && (u < nB || u >= U()); }
+  __device__ bool shared(int u) const { return existsB && (u < nC || u >= U()); }
+  __device__ bool centroid(int u) const { return u >= U(); }
+};
+
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  return (static_cast<uint64_t>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 
 template <int D, int KB>
 __global__ void __launch_bounds__(kFusedThreads, 1)
@@ -64,149 +103,211 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   using Lay = FusedLayout<D>;
   constexpr int QT = Lay::QT, G = QT / KB, CB = D / 64, NS = kFusedStages;
   constexpr uint32_t SLOT = Lay::kSlot;
-  constexpr uint32_t OC = 256, QHC = 256 + D;
+  constexpr uint32_t OC = 256;  // O_A at OC, O_B at OC + D
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sRing = smem + Lay::kQ;
+  uint8_t* sQ = smem;  // [2][kQ]
+  uint8_t* sRing = smem + 2 * Lay::kQ;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sRing + Lay::kRing);
   uint64_t* full = bars;
   uint64_t* empty = bars + NS;
-  uint64_t* q_full = bars + 2 * NS;
-  uint64_t* s_full = q_full + 1;  // [2]
-  uint64_t* p_full = s_full + 2;  // [2]
-  uint64_t* o_done = p_full + 2;
-  uint64_t* o_final = o_done + 1;
-  uint64_t* mma_idle = o_final + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + 8);
+  uint64_t* q_full = bars + 2 * NS;      // [2]
+  uint64_t* q_empty = q_full + 2;        // [2]
+  uint64_t* s_full = q_empty + 2;        // [2]
+  uint64_t* p_full = s_full + 2;         // [2]
+  uint64_t* o_final = p_full + 2;        // [2]
+  uint64_t* epi_done = o_final + 2;      // [2]
+  uint64_t* list_full = epi_done + 2;    // [2]
+  uint64_t* list_empty = list_full + 2;  // [2]
+  uint64_t* mma_idle = list_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Lay::kNumBars);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* n_exact_s = reinterpret_cast<int*>(tmem_slot + 2);
-  int* list = reinterpret_cast<int*>(tmem_slot + 4);
+  int* lists = reinterpret_cast<int*>(tmem_slot + 4);
   const int words = a.nbp / 32;
-  uint32_t* mask = reinterpret_cast<uint32_t*>(list + G * a.kk);
+  const int list_stride = (int)Lay::list_ints(G, a.kk, words);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int qt = blockIdx.x, bh = blockIdx.y;
   const int nb = a.nb;
+  const int n_cent = a.nbp / 128;
+  const int pairs_per_head = (a.n_qtiles + 1) / 2;
 
-  // ------------------------------------------------------------ set-up
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(q_full, 1);
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
-    mbar_init(&p_full[0], 128);
-    mbar_init(&p_full[1], 128);
-    mbar_init(o_done, 1);
-    mbar_init(o_final, 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&q_full[x], 1);
+      mbar_init(&q_empty[x], 1);
+      mbar_init(&s_full[x], 1);
+      mbar_init(&p_full[x], 128);
+      mbar_init(&o_final[x], 1);
+      mbar_init(&epi_done[x], 128);
+      mbar_init(&list_full[x], 1);
+      mbar_init(&list_empty[x], 9);
+    }
     mbar_init(mma_idle, 1);
     *abort = 0;
     fence_mbar_init();
   }
-  if (warp == 4 && lane == 0) {
-    prefetch_tensormap(&tmQ);
-    prefetch_tensormap(&tmK);
-    prefetch_tensormap(&tmV);
-    prefetch_tensormap(&tmKc);
-    prefetch_tensormap(&tmVc);
-    prefetch_tensormap(&tmH);
-  }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
-  }
-  for (int e = threadIdx.x; e < G * words; e += blockDim.x) mask[e] = 0u;
-  __syncthreads();
-  for (int g = 0; g < G; ++g) {
-    const int i = qt * G + g;
-    if (i >= nb) continue;
-    const int32_t* si = a.sel + ((size_t)bh * nb + i) * a.kk;
-    for (int e = threadIdx.x; e < a.kk; e += blockDim.x) {
-      const int j = si[e];
-      if (j < 0 || j >= nb) {
-        raise_device_error(PISA_ERR_DEVICE_CHECK);
-      } else {
-        atomicOr(&mask[g * words + (j >> 5)], 1u << (j & 31));
-      }
-    }
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    // exact tiles: ascending union of the selected blocks, with group bits
-    int n = 0;
-    for (int w = 0; w < words; ++w) {
-      uint32_t any = 0;
-#pragma unroll
-      for (int g = 0; g < G; ++g) any |= mask[g * words + w];
-      while (any) {
-        const int b = __ffs(any) - 1;
-        any &= any - 1;
-        int gm = 0;
-#pragma unroll
-        for (int g = 0; g < G; ++g) gm |= ((mask[g * words + w] >> b) & 1u) << g;
-        list[n++] = (w * 32 + b) | (gm << 24);
-      }
-    }
-    *n_exact_s = n;
   }
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  const int n_exact = *n_exact_s;
-  const int n_cent = a.nbp / 128;
-  const int n_t = n_exact + n_cent;
 
-  if (warp == 4) {
-    // -------------------------------------------------------- TMA producer
+  // Register split within the 384 x 168 registers the CTA is launched with:
+  // the third warpgroup drops to 104, the softmax warpgroups rise to 200,
+  // 2 x 128 x 200 + 128 x 104 = 64512 = 384 x 168 (an increase beyond the
+  // launch total would wait forever).
+  if (warp >= 8) {
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 104;\n" ::: "memory");
+   if (warp == 8) {
+    // ================================================================ producer
     if (lane == 0) {
-      mbar_expect_tx(q_full, Lay::kQ);
-#pragma unroll
-      for (int cb = 0; cb < CB; ++cb) tma_load_3d(sQ + cb * QT * 128, &tmQ, q_full, cb * 64, qt * QT, bh);
-      int it = 0;
-      auto load = [&](const CUtensorMap* map, int row, int rows) -> bool {
-        const int s = it % NS;
-        const uint32_t ph = (it / NS) & 1;
-        if (!mbar_wait(&empty[s], ph ^ 1, abort)) return false;
-        mbar_expect_tx(&full[s], rows * D * 2);
-#pragma unroll
-        for (int cb = 0; cb < CB; ++cb) tma_load_3d(sRing + s * SLOT + cb * rows * 128, map, &full[s], cb * 64, row, bh);
-        ++it;
-        return true;
-      };
-      auto loadK = [&](int t) -> bool {
-        if (t < n_exact) return load(&tmK, (list[t] & 0xFFFFFF) * KB, KB);
-        const int c = t - n_exact;
-        return load(&tmKc, c * 128, 128) && load(&tmKc, a.nbp + c * 128, 128);
-      };
-      auto loadV = [&](int t) -> bool {
-        if (t < n_exact) return load(&tmV, (list[t] & 0xFFFFFF) * KB, KB);
-        const int c = t - n_exact;
-        return load(&tmVc, c * 128, 128) && load(&tmVc, a.nbp + c * 128, 128);
-      };
-      bool ok = load(&tmH, 0, D) && load(&tmH, D, D);
-      for (int t = 0; ok && t < n_t; ++t) ok = loadK(t) && (t == 0 || loadV(t - 1));
-      if (ok) ok = loadV(n_t - 1);
-      if (!ok) {
-        // let the copies already issued land before the CTA can exit
-        const int first = it > NS ? it - NS : 0;
-        for (int u = first; u < it; ++u) mbar_wait(&full[u % NS], (u / NS) & 1, abort);
-      }
+      prefetch_tensormap(&tmQ);
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      prefetch_tensormap(&tmKc);
+      prefetch_tensormap(&tmVc);
+      prefetch_tensormap(&tmH);
     }
-  } else if (warp == 5) {
-    // -------------------------------------------------------- MMA issuer
+    int it = 0, qloads[2] = {0, 0};
+    bool ok = true;
+    int lp = 0;
+    for (int p = blockIdx.x; ok && p < a.n_pairs; p += gridDim.x, ++lp) {
+      const int slot = lp & 1;
+      int* L_ = lists + slot * list_stride;
+      int* eA = L_ + 8;
+      int* eB = eA + G * a.kk;
+      uint32_t* mA = reinterpret_cast<uint32_t*>(eB + G * a.kk);
+      uint32_t* mB = mA + G * words;
+      if (!__all_sync(0xffffffffu, mbar_wait(&list_empty[slot], ((lp >> 1) & 1) ^ 1, abort))) {
+        ok = false;
+        break;
+      }
+      const int bh = p / pairs_per_head;
+      const int tA = 2 * (p % pairs_per_head);
+      const int existsB = (tA + 1) < a.n_qtiles;
+      for (int e = lane; e < 2 * G * words; e += 32) mA[e] = 0u;
+      __syncwarp();
+      for (int x = 0; x < 1 + existsB; ++x) {
+        uint32_t* mX = x ? mB : mA;
+        for (int g = 0; g < G; ++g) {
+          const int i = (tA + x) * G + g;
+          if (i >= nb) continue;
+          const int32_t* si = a.sel + ((size_t)bh * nb + i) * a.kk;
+          for (int e = lane; e < a.kk; e += 32) {
+            const int j = si[e];
+            if (j < 0 || j >= nb) {
+              raise_device_error(PISA_ERR_DEVICE_CHECK);
+            } else {
+              atomicOr(&mX[g * words + (j >> 5)], 1u << (j & 31));
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) {
+        int nA = 0, nB = 0, nC = 0;
+        // pass 0: blocks of both tiles; pass 1: A only; pass 2: B only
+        for (int pass = 0; pass < 3; ++pass) {
+          for (int w = 0; w < words; ++w) {
+            uint32_t uA = 0, uB = 0;
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+              uA |= mA[g * words + w];
+              uB |= mB[g * words + w];
+            }
+            uint32_t bits = pass == 0 ? (uA & uB) : pass == 1 ? (uA & ~uB) : (uB & ~uA);
+            while (bits) {
+              const int b = __ffs(bits) - 1;
+              bits &= bits - 1;
+              int gA = 0, gB = 0;
+#pragma unroll
+              for (int g = 0; g < G; ++g) {
+                gA |= ((mA[g * words + w] >> b) & 1u) << g;
+                gB |= ((mB[g * words + w] >> b) & 1u) << g;
+              }
+              const int j = w * 32 + b;
+              if (pass != 2) eA[nA++] = j | (gA << 24);
+              if (pass != 1) eB[nB++] = j | (gB << 24);
+              if (pass == 0) ++nC;
+            }
+          }
+        }
+        L_[0] = nA;
+        L_[1] = nB;
+        L_[2] = nC;
+        L_[3] = existsB;
+        L_[4] = bh;
+        L_[5] = tA;
+        mbar_arrive(&list_full[slot]);
+
+        const PairPlan pl{nA, nB, nC, existsB, n_cent};
+        auto load = [&](const CUtensorMap* map, int row, int rows) -> bool {
+          const int s = it % NS;
+          if (!mbar_wait(&empty[s], ((it / NS) & 1) ^ 1, abort)) return false;
+          mbar_expect_tx(&full[s], rows * D * 2);
+#pragma unroll
+          for (int cb = 0; cb < CB; ++cb)
+            tma_load_3d(sRing + s * SLOT + cb * rows * 128, map, &full[s], cb * 64, row, bh);
+          ++it;
+          return true;
+        };
+        auto loadK = [&](int x, int u) -> bool {
+          if (!pl.centroid(u)) return load(&tmK, ((x ? eB : eA)[u] & 0xFFFFFF) * KB, KB);
+          const int c = u - pl.U();
+          return load(&tmKc, c * 128, 128) && load(&tmKc, a.nbp + c * 128, 128);
+        };
+        auto loadV = [&](int x, int u) -> bool {
+          if (!pl.centroid(u)) return load(&tmV, ((x ? eB : eA)[u] & 0xFFFFFF) * KB, KB);
+          const int c = u - pl.U();
+          return load(&tmVc, c * 128, 128) && load(&tmVc, a.nbp + c * 128, 128);
+        };
+        for (int x = 0; ok && x < 1 + existsB; ++x) {
+          ok = mbar_wait(&q_empty[x], (qloads[x] & 1) ^ 1, abort);
+          if (!ok) break;
+          mbar_expect_tx(&q_full[x], Lay::kQ);
+#pragma unroll
+          for (int cb = 0; cb < CB; ++cb)
+            tma_load_3d(sQ + x * Lay::kQ + cb * QT * 128, &tmQ, &q_full[x], cb * 64, (tA + x) * QT, bh);
+          ++qloads[x];
+        }
+        const int T = pl.T();
+        if (ok) ok = loadK(0, 0);
+        if (ok && pl.activeB(0) && !pl.shared(0)) ok = loadK(1, 0);
+        for (int u = 0; ok && u < T; ++u) {
+          if (pl.activeA(u)) ok = loadV(0, u);
+          if (ok && u + 1 < T && pl.activeA(u + 1)) ok = loadK(0, u + 1);
+          if (ok && pl.activeB(u) && !pl.shared(u)) ok = loadV(1, u);
+          if (ok && u + 1 < T && pl.activeB(u + 1) && !pl.shared(u + 1)) ok = loadK(1, u + 1);
+        }
+        if (ok) ok = load(&tmH, 0, D) && load(&tmH, D, D);
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    }
+    if (!ok && lane == 0) {
+      // let the copies already issued land before the CTA can exit
+      const int first = it > NS ? it - NS : 0;
+      for (int u = first; u < it; ++u) mbar_wait(&full[u % NS], (u / NS) & 1, abort);
+    }
+   } else if (warp == 9) {
+    // ================================================================ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(128, KB, false, false);
       constexpr uint32_t idC = idesc_bf16(128, 128, false, false);
       constexpr uint32_t idH = idesc_bf16(128, D, false, false);
       constexpr uint32_t idO = idesc_bf16(128, D, false, true);
-      const uint32_t qaddr = smem_u32(sQ);
       const uint32_t ring = smem_u32(sRing);
-      auto qdesc = [&](int kk) { return desc_sw128(qaddr + (kk >> 2) * QT * 128 + (kk & 3) * 32, 16, 1024); };
+      const uint32_t qbase = smem_u32(sQ);
+      auto qdesc = [&](int x, int kk) {
+        return desc_sw128(qbase + x * Lay::kQ + (kk >> 2) * QT * 128 + (kk & 3) * 32, 16, 1024);
+      };
       auto kdesc = [&](int s, int rows, int kk) {
         return desc_sw128(ring + s * SLOT + (kk >> 2) * rows * 128 + (kk & 3) * 32, 16, 1024);
       };
@@ -221,217 +322,292 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         ++it;
         return true;
       };
-      auto pv = [&](int u) -> bool {
-        const int buf = u & 1;
-        if (!mbar_wait(&p_full[buf], (u >> 1) & 1, abort)) return false;
+      int qwaits[2] = {0, 0}, steps[2] = {0, 0}, epis[2] = {0, 0};
+      bool ok = true;
+      int lp = 0;
+      for (int p = blockIdx.x; ok && p < a.n_pairs; p += gridDim.x, ++lp) {
+        const int slot = lp & 1;
+        if (!(ok = mbar_wait(&list_full[slot], (lp >> 1) & 1, abort))) break;
+        const int* L_ = lists + slot * list_stride;
+        const PairPlan pl{L_[0], L_[1], L_[2], L_[3], n_cent};
+        const int T = pl.T();
+        for (int x = 0; ok && x < 1 + pl.existsB; ++x) {
+          ok = mbar_wait(&q_full[x], qwaits[x] & 1, abort);
+          ++qwaits[x];
+        }
+        if (!ok) break;
         fence_after_sync();
-        const uint32_t pa = tmem + buf * 128;
-        if (u < n_exact) {
-          int s;
-          if (!take(s)) return false;
-          for (int kk = 0; kk < KB / 16; ++kk)
-            mma_ts(tmem + OC, pa + kk * 8, vdesc(s, KB, kk), idO, (u > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&empty[s]);
-        } else {
-          int s1, s2;
-          if (!take(s1) || !take(s2)) return false;
-          for (int kk = 0; kk < 8; ++kk) mma_ts(tmem + OC, pa + kk * 8, vdesc(s1, 128, kk), idO, 1u);
-          for (int kk = 0; kk < 8; ++kk) mma_ts(tmem + OC, pa + kk * 8, vdesc(s2, 128, kk), idO, 1u);
-          mma_commit(&empty[s1]);
-          mma_commit(&empty[s2]);
+        int ks[2] = {-1, -1}, vs[2] = {-1, -1};  // slots of the last K / V items
+        bool first_pv[2] = {true, true};
+        auto issue_s = [&](int x, int u) -> bool {
+          const uint32_t sc = tmem + x * 128;
+          if (!((x == 1) && pl.shared(u))) {  // tile B reuses tile A's items when shared
+            if (!pl.centroid(u)) {
+              if (!take(ks[0])) return false;
+              ks[1] = -1;
+            } else if (!take(ks[0]) || !take(ks[1])) {
+              return false;
+            }
+          }
+          if (!pl.centroid(u)) {
+            for (int kk = 0; kk < D / 16; ++kk) mma_ss(sc, qdesc(x, kk), kdesc(ks[0], KB, kk), idS, kk > 0 ? 1u : 0u);
+          } else {
+            for (int kk = 0; kk < D / 16; ++kk) mma_ss(sc, qdesc(x, kk), kdesc(ks[0], 128, kk), idC, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) mma_ss(sc, qdesc(x, kk), kdesc(ks[1], 128, kk), idC, 1u);
+          }
+          if (!((x == 0) && pl.shared(u))) {
+            mma_commit(&empty[ks[0]]);
+            if (ks[1] >= 0) mma_commit(&empty[ks[1]]);
+          }
+          mma_commit(&s_full[x]);
+          return true;
+        };
+        auto issue_pv = [&](int x, int u) -> bool {
+          if (!mbar_wait(&p_full[x], steps[x] & 1, abort)) return false;
+          ++steps[x];
+          fence_after_sync();
+          const uint32_t pa = tmem + x * 128;
+          const uint32_t oc = tmem + OC + x * D;
+          if (!((x == 1) && pl.shared(u))) {
+            if (!pl.centroid(u)) {
+              if (!take(vs[0])) return false;
+              vs[1] = -1;
+            } else if (!take(vs[0]) || !take(vs[1])) {
+              return false;
+            }
+          }
+          if (!pl.centroid(u)) {
+            for (int kk = 0; kk < KB / 16; ++kk)
+              mma_ts(oc, pa + kk * 8, vdesc(vs[0], KB, kk), idO, (!first_pv[x] || kk > 0) ? 1u : 0u);
+          } else {
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ts(oc, pa + kk * 8, vdesc(vs[0], 128, kk), idO, (!first_pv[x] || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 8; ++kk) mma_ts(oc, pa + kk * 8, vdesc(vs[1], 128, kk), idO, 1u);
+          }
+          first_pv[x] = false;
+          if (!((x == 0) && pl.shared(u))) {
+            mma_commit(&empty[vs[0]]);
+            if (vs[1] >= 0) mma_commit(&empty[vs[1]]);
+          }
+          return true;
+        };
+        // before reusing S_x / O_x the previous epilogue of tile x must have read them
+        auto epi_wait = [&](int x) -> bool {
+          if (epis[x] == 0) return true;
+          if (!mbar_wait(&epi_done[x], (epis[x] - 1) & 1, abort)) return false;
+          fence_after_sync();
+          return true;
+        };
+        ok = epi_wait(0) && issue_s(0, 0);
+        if (ok && pl.activeB(0)) ok = epi_wait(1) && issue_s(1, 0);
+        for (int u = 0; ok && u < T; ++u) {
+          if (pl.activeA(u)) ok = issue_pv(0, u);
+          if (ok && u + 1 < T && pl.activeA(u + 1)) ok = issue_s(0, u + 1);
+          if (ok && pl.activeB(u)) ok = issue_pv(1, u);
+          if (ok && u + 1 < T && pl.activeB(u + 1)) ok = issue_s(1, u + 1);
         }
-        mma_commit(o_done);
-        return true;
-      };
-      bool ok = mbar_wait(q_full, 0, abort);
-      if (ok) {
-        fence_after_sync();
-        int sh, sl;
-        ok = take(sh) && take(sl);
-        if (ok) {
-          for (int kk = 0; kk < D / 16; ++kk) mma_ss(tmem + QHC, qdesc(kk), kdesc(sh, D, kk), idH, kk > 0 ? 1u : 0u);
-          for (int kk = 0; kk < D / 16; ++kk) mma_ss(tmem + QHC, qdesc(kk), kdesc(sl, D, kk), idH, 1u);
-          mma_commit(&empty[sh]);
-          mma_commit(&empty[sl]);
+        if (!ok) break;
+        // first-order term q Hbar into each tile's S columns; then Q and Hbar are free
+        int h0, h1;
+        if (!(ok = take(h0) && take(h1))) break;
+        for (int x = 0; x < 1 + pl.existsB; ++x) {
+          const uint32_t sc = tmem + x * 128;
+          for (int kk = 0; kk < D / 16; ++kk) mma_ss(sc, qdesc(x, kk), kdesc(h0, D, kk), idH, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) mma_ss(sc, qdesc(x, kk), kdesc(h1, D, kk), idH, 1u);
+          mma_commit(&o_final[x]);
+          mma_commit(&q_empty[x]);
+          ++epis[x];
         }
+        mma_commit(&empty[h0]);
+        mma_commit(&empty[h1]);
+        mbar_arrive(&list_empty[slot]);
       }
-      for (int t = 0; ok && t < n_t; ++t) {
-        const uint32_t sc = tmem + (t & 1) * 128;
-        if (t < n_exact) {
-          int s;
-          ok = take(s);
-          if (!ok) break;
-          for (int kk = 0; kk < D / 16; ++kk) mma_ss(sc, qdesc(kk), kdesc(s, KB, kk), idS, kk > 0 ? 1u : 0u);
-          mma_commit(&empty[s]);
-        } else {
-          int s1, s2;
-          ok = take(s1) && take(s2);
-          if (!ok) break;
-          for (int kk = 0; kk < D / 16; ++kk) mma_ss(sc, qdesc(kk), kdesc(s1, 128, kk), idC, kk > 0 ? 1u : 0u);
-          for (int kk = 0; kk < D / 16; ++kk) mma_ss(sc, qdesc(kk), kdesc(s2, 128, kk), idC, 1u);
-          mma_commit(&empty[s1]);
-          mma_commit(&empty[s2]);
-        }
-        mma_commit(&s_full[t & 1]);
-        if (t >= 1) ok = pv(t - 1);
-      }
-      if (ok) ok = pv(n_t - 1);
-      if (ok) mma_commit(o_final);
-      // nothing of ours may still run on the tensor cores when TMEM is freed
       mma_commit(mma_idle);
       volatile int never = 0;
       mbar_wait(mma_idle, 0, &never);
     }
     __syncwarp();
+   }
   } else {
-    // -------------------------------------------------------- softmax warps 0-3
-    const int row = threadIdx.x;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 200;\n" ::: "memory");
+    // ================================================================ softmax: tile A (warps 0-3), B (4-7)
+    const int x = warp / 4;
+    const int row = threadIdx.x % 128;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
+    const uint32_t sbase = lane_base + x * 128;
+    const uint32_t obase = lane_base + OC + x * D;
     const int g = row / KB;
-    const int qrow = qt * QT + row;
     const float c2 = a.scale_log2;
     const int n_tail = a.L - (nb - 1) * a.block;
-    float m = -INFINITY, l = 0.f, beta = 0.f;
-    uint32_t s[128];
+    int steps = 0, finals = 0;
     bool ok = true;
-    for (int t = 0; t < n_t; ++t) {
-      const int buf = t & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[buf], (t >> 1) & 1, abort))) {
+    int lp = 0;
+    for (int p = blockIdx.x; ok && p < a.n_pairs; p += gridDim.x, ++lp) {
+      const int slot = lp & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&list_full[slot], (lp >> 1) & 1, abort))) {
         ok = false;
         break;
       }
-      fence_after_sync();
-      const uint32_t sa = lane_base + buf * 128;
-      const bool exact = t < n_exact;
-      float tmax = -INFINITY;
-      float x_tail = -INFINITY;
-      if (exact) {
-        tmem_ld32(sa, s);
-        if (KB == 128) {
-          tmem_ld32(sa + 32, s + 32);
-          tmem_ld32(sa + 64, s + 64);
-          tmem_ld32(sa + 96, s + 96);
-        } else {
-          tmem_ld32(sa + 32, s + 32);
-        }
-        tmem_wait_ld();
-        const int e = list[t];
-        const int j = e & 0xFFFFFF;
-        const int nvalid = ((e >> (24 + g)) & 1) ? min(KB, a.L - j * KB) : 0;
-#pragma unroll
-        for (int c = 0; c < KB; ++c) {
-          const float x = c < nvalid ? __uint_as_float(s[c]) * c2 : -INFINITY;
-          s[c] = __float_as_uint(x);
-          tmax = fmaxf(tmax, x);
-        }
-      } else {
-        tmem_ld32(sa, s);
-        tmem_ld32(sa + 32, s + 32);
-        tmem_ld32(sa + 64, s + 64);
-        tmem_ld32(sa + 96, s + 96);
-        tmem_wait_ld();
-        const int c0 = (t - n_exact) * 128;
-        const uint32_t* mw = mask + g * words + c0 / 32;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const uint32_t bits = mw[w];
-#pragma unroll
-          for (int b = 0; b < 32; ++b) {
-            const int c = w * 32 + b;
-            const bool use = (c0 + c < nb) && !((bits >> b) & 1u);
-            const float x = use ? __uint_as_float(s[c]) * c2 : -INFINITY;
-            s[c] = __float_as_uint(x);
-            tmax = fmaxf(tmax, x);
-            if (c0 + c == nb - 1) x_tail = x;
+      const int* L_ = lists + slot * list_stride;
+      const PairPlan pl{L_[0], L_[1], L_[2], L_[3], n_cent};
+      const int bh = L_[4];
+      const int qtile = L_[5] + x;
+      const int* ent = L_ + 8 + x * G * a.kk;
+      const uint32_t* msk = reinterpret_cast<const uint32_t*>(L_ + 8 + 2 * G * a.kk) + x * G * words + g * words;
+      if (x == 0 || pl.existsB) {
+        const int qrow = qtile * QT + row;
+        const int T = pl.T();
+        float m = -INFINITY, l = 0.f, beta = 0.f;
+        uint32_t s[128];
+        for (int u = 0; u < T; ++u) {
+          if (!(x == 0 ? pl.activeA(u) : pl.activeB(u))) continue;
+          if (!__all_sync(0xffffffffu, mbar_wait(&s_full[x], steps & 1, abort))) {
+            ok = false;
+            break;
           }
+          ++steps;
+          fence_after_sync();
+          const bool exact = !pl.centroid(u);
+          float tmax = -INFINITY, x_tail = -INFINITY;
+          int ncols = 128;
+          if (exact) {
+            ncols = KB;
+            tmem_ld32(sbase, s);
+            tmem_ld32(sbase + 32, s + 32);
+            if (KB == 128) {
+              tmem_ld32(sbase + 64, s + 64);
+              tmem_ld32(sbase + 96, s + 96);
+            }
+            tmem_wait_ld();
+            const int e = ent[u];
+            const int j = e & 0xFFFFFF;
+            const int nvalid = ((e >> (24 + g)) & 1) ? min(KB, a.L - j * KB) : 0;
+            if (__all_sync(0xffffffffu, nvalid == KB)) {
+#pragma unroll
+              for (int c = 0; c < KB; ++c) tmax = fmaxf(tmax, __uint_as_float(s[c]));
+            } else {
+#pragma unroll
+              for (int c = 0; c < KB; ++c) {
+                const float v = c < nvalid ? __uint_as_float(s[c]) : -INFINITY;
+                s[c] = __float_as_uint(v);
+                tmax = fmaxf(tmax, v);
+              }
+            }
+          } else {
+            tmem_ld32(sbase, s);
+            tmem_ld32(sbase + 32, s + 32);
+            tmem_ld32(sbase + 64, s + 64);
+            tmem_ld32(sbase + 96, s + 96);
+            tmem_wait_ld();
+            const int c0 = (u - pl.U()) * 128;
+            const uint32_t* mw = msk + c0 / 32;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const uint32_t bits = mw[w];
+#pragma unroll
+              for (int b = 0; b < 32; ++b) {
+                const int c = w * 32 + b;
+                const bool use = (c0 + c < nb) && !((bits >> b) & 1u);
+                const float v = use ? __uint_as_float(s[c]) : -INFINITY;
+                s[c] = __float_as_uint(v);
+                tmax = fmaxf(tmax, v);
+                if (c0 + c == nb - 1) x_tail = v;
+              }
+            }
+          }
+          // running max in log2 units; lazy rescale when it grows by more than 8
+          const float m_new = fmaxf(m, tmax * c2);
+          float f = 1.f;
+          if (m_new > m + 8.f) {
+            if (m != -INFINITY) {
+              f = ex2(m - m_new);
+              l *= f;
+              beta *= f;
+            }
+            m = m_new;
+          }
+          // O is quiescent here: this step's S MMA was issued after the previous
+          // PV of this tile, so that PV has completed.
+          if (__any_sync(0xffffffffu, f != 1.f)) {
+            uint32_t o[32];
+#pragma unroll 1
+            for (int ch = 0; ch < D / 32; ++ch) {
+              tmem_ld32(obase + ch * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+              tmem_st32(obase + ch * 32, o);
+            }
+            tmem_wait_st();
+          }
+          const float mu = (m == -INFINITY) ? 0.f : m;
+          const uint64_t c2x2 = f2_pack(c2, c2), nmu = f2_pack(-mu, -mu);
+          uint64_t acc = 0;
+#pragma unroll
+          for (int c = 0; c < 128; c += 2) {
+            if (c < ncols) {
+              const uint64_t t = ffma2(f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), c2x2, nmu);
+              const float p0 = ex2(f2_lo(t));
+              const float p1 = ex2(f2_hi(t));
+              acc = fadd2(acc, f2_pack(p0, p1));
+              s[c >> 1] = pack_bf16x2(p0, p1);
+            }
+          }
+          const float sum = f2_lo(acc) + f2_hi(acc);
+          if (exact) {
+            l += sum;
+          } else {
+            beta += sum;
+            l += (float)a.block * sum;
+            if (x_tail != -INFINITY) l += (float)(n_tail - a.block) * ex2(x_tail * c2 - mu);
+          }
+          tmem_st32(sbase, s);
+          if (ncols == 128) tmem_st32(sbase + 32, s + 32);
+          tmem_wait_st();
+          fence_before_sync();
+          mbar_arrive(&p_full[x]);
         }
-      }
-      // lazy rescale: move the reference max only when it grows by > 2^8
-      const float m_new = fmaxf(m, tmax);
-      float f = 1.f;
-      if (m_new > m + 8.f) {
-        if (m != -INFINITY) {
-          f = ex2(m - m_new);
-          l *= f;
-          beta *= f;
-        }
-        m = m_new;
-      }
-      const bool rescale_o = (f != 1.f) && t >= 1;
-      if (__any_sync(0xffffffffu, rescale_o)) {
-        if (!__all_sync(0xffffffffu, mbar_wait(o_done, (t - 1) & 1, abort))) {
+        if (!ok) break;
+        // epilogue: o = (O + s beta q Hbar) / l, q Hbar in this tile's S columns
+        if (!__all_sync(0xffffffffu, mbar_wait(&o_final[x], finals & 1, abort))) {
           ok = false;
           break;
         }
+        ++finals;
         fence_after_sync();
-        uint32_t o[32];
+        const float inv = 1.f / l;
+        const float fo = a.scale * beta;
+        __nv_bfloat16* dst = a.out + ((size_t)bh * a.L + qrow) * D;
 #pragma unroll 1
         for (int ch = 0; ch < D / 32; ++ch) {
-          tmem_ld32(lane_base + OC + ch * 32, o);
+          uint32_t o[32], h[32];
+          tmem_ld32(obase + ch * 32, o);
+          tmem_ld32(sbase + ch * 32, h);
           tmem_wait_ld();
+          uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-          tmem_st32(lane_base + OC + ch * 32, o);
-        }
-        tmem_wait_st();
-      }
-      const float mu = (m == -INFINITY) ? 0.f : m;
-      float sum = 0.f;
-      const int ncols = exact ? KB : 128;
+          for (int e = 0; e < 16; ++e) {
+            const float y0 = fmaf(fo, __uint_as_float(h[2 * e]), __uint_as_float(o[2 * e])) * inv;
+            const float y1 = fmaf(fo, __uint_as_float(h[2 * e + 1]), __uint_as_float(o[2 * e + 1])) * inv;
+            pk[e] = pack_bf16x2(y0, y1);
+          }
+          if (qrow < a.L) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + ch * 32);
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        if (c < ncols) {
-          const float p0 = ex2(__uint_as_float(s[c]) - mu);
-          const float p1 = ex2(__uint_as_float(s[c + 1]) - mu);
-          sum += p0 + p1;
-          s[c >> 1] = pack_bf16x2(p0, p1);
+            for (int e = 0; e < 4; ++e) d4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          }
         }
+        fence_before_sync();
+        mbar_arrive(&epi_done[x]);
       }
-      if (exact) {
-        l += sum;
-      } else {
-        beta += sum;
-        l += (float)a.block * sum;
-        if (x_tail != -INFINITY) l += (float)(n_tail - a.block) * ex2(x_tail - mu);
-      }
-      tmem_st32(sa, s);
-      if (ncols == 128) tmem_st32(sa + 32, s + 32);
-      tmem_wait_st();
-      fence_before_sync();
-      mbar_arrive(&p_full[buf]);
-    }
-    // epilogue: o_t = (O + s beta q Hbar) / l
-    if (ok && __all_sync(0xffffffffu, mbar_wait(o_final, 0, abort))) {
-      fence_after_sync();
-      const float inv = 1.f / l;
-      const float fo = a.scale * beta;
-      __nv_bfloat16* dst = a.out + ((size_t)bh * a.L + qrow) * D;
-#pragma unroll 1
-      for (int ch = 0; ch < D / 32; ++ch) {
-        uint32_t o[32], h[32];
-        tmem_ld32(lane_base + OC + ch * 32, o);
-        tmem_ld32(lane_base + QHC + ch * 32, h);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float y0 = (__uint_as_float(o[2 * e]) + fo * __uint_as_float(h[2 * e])) * inv;
-          const float y1 = (__uint_as_float(o[2 * e + 1]) + fo * __uint_as_float(h[2 * e + 1])) * inv;
-          pk[e] = pack_bf16x2(y0, y1);
-        }
-        if (qrow < a.L) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + ch * 32);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) d4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-        }
-      }
+      if (lane == 0) mbar_arrive(&list_empty[slot]);
     }
   }
 
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
-  if (warp == 5) tmem_dealloc(tmem, 512);
+  if (warp == 9) tmem_dealloc(tmem, 512);
 }
 
 // Centroid and Hbar operands in the fused kernel's bf16 hi/lo format:

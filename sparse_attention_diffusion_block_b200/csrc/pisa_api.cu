@@ -280,7 +280,14 @@ pisa_status run_fused_sm100(const __nv_bfloat16* q, const __nv_bfloat16* k, cons
   fa.block = s.block;
   fa.scale = 1.0f / sqrtf((float)D);
   fa.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
-  fused_sm100_kernel<D, KB><<<dim3((s.L + 127) / 128, BH), kFusedThreads, smem, st>>>(mQ, mK, mV, mKc, mVc, mH, fa);
+  fa.n_qtiles = (s.L + 127) / 128;
+  fa.n_pairs = BH * ((fa.n_qtiles + 1) / 2);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return PISA_ERR_CUDA;
+  const int grid = fa.n_pairs < sms ? fa.n_pairs : sms;
+  fused_sm100_kernel<D, KB><<<grid, kFusedThreads, smem, st>>>(mQ, mK, mV, mKc, mVc, mH, fa);
   return last_launch();
 }
 
