@@ -1,6 +1,7 @@
 """Builds libpisa.so in-tree with nvcc for sm_100a (B200).
 
-Usage: python -m sparse_attention_diffusion_block_b200.build [--force]
+Usage: python sparse_attention_diffusion_block_b200/build.py [--force]
+(run it by path: importing the package needs the library this builds)
 """
 
 from __future__ import annotations
