@@ -146,6 +146,41 @@ pisa_status pisa_attn_fwd(const void* q, const void* k, const void* v, void* out
                           float keep_ratio, void* workspace, size_t workspace_bytes,
                           void* stream);
 
+/* Size in bytes of the fixed device scratch array used by
+ * pisa_attn_fwd_with_sel_noalloc (32 MiB). */
+#define PISA_NOALLOC_SCRATCH_BYTES (32ull * 1024ull * 1024ull)
+
+/* pisa_attn_fwd_with_sel for callers that cannot allocate device memory: code
+ * that is handed only its input and output buffers (a plugin inside another
+ * framework's memory pool, a pre-allocated serving runtime, a captured
+ * sequence that forbids cudaMalloc), where no workspace can be created.  The
+ * paper has no counterpart; this is an interface convenience.
+ *
+ * Same arguments and results as pisa_attn_fwd_with_sel minus the workspace.
+ * The scratch that pisa_attn_fwd_with_sel takes from the caller's workspace
+ * (the tensor-core kernel's bf16 hi/lo copies of kbar, vsum and Hbar) lives
+ * instead in one device array of PISA_NOALLOC_SCRATCH_BYTES compiled into the
+ * library; every GPU that loads the library holds that memory until the
+ * process exits.
+ *   - A call whose scratch need, pisa_fused_workspace_size(batch, heads, L, d,
+ *     block), exceeds PISA_NOALLOC_SCRATCH_BYTES is rejected with
+ *     PISA_ERR_WORKSPACE before anything is launched.
+ *   - It calls no allocating routine (no cudaMalloc, cudaFree or library
+ *     allocator).
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - All calls share the one array, which keeps what the last call wrote.
+ *     Each call rewrites every scratch byte it later reads, so nothing needs
+ *     to start at zero; but calls that overlap on the GPU (other streams,
+ *     other host threads) race on the array and must be serialised by the
+ *     caller. */
+pisa_status pisa_attn_fwd_with_sel_noalloc(const void* q, const void* k, const void* v, void* out,
+                                           pisa_dtype dtype, int batch, int heads, int L, int d,
+                                           int block, const float* kbar, const float* vsum,
+                                           const float* hbar, const int32_t* sel, int k_sel,
+                                           void* stream);
+
 /* Reads (and, when reset != 0, clears) the device error word that bounded
  * waits and index checks set.  Synchronises `stream`.  Returns PISA_OK,
  * PISA_ERR_TIMEOUT, PISA_ERR_DEVICE_CHECK or PISA_ERR_CUDA. */

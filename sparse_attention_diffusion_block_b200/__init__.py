@@ -7,7 +7,7 @@ loudly when the library has not been built.
 
 Entry points mirror the C names (without the ``pisa_`` prefix):
 block_stats, cov_norm, block_first_order, select, attn_fwd_with_sel, attn_fwd,
-keep_count, workspace_size, stats_workspace_size, fused_workspace_size,
+attn_fwd_with_sel_noalloc, keep_count, workspace_size, stats_workspace_size, fused_workspace_size,
 device_status, status_string.
 """
 
@@ -38,12 +38,13 @@ PISA_ERR_TIMEOUT = -5
 PISA_ERR_DEVICE_CHECK = -6
 PISA_BF16 = 0
 PISA_FP32 = 1
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # PISA_NOALLOC_SCRATCH_BYTES
 
 EXPORTS = (
     "pisa_status_string", "pisa_keep_count", "pisa_stats_workspace_size",
     "pisa_fused_workspace_size", "pisa_workspace_size", "pisa_block_stats", "pisa_cov_norm",
     "pisa_block_first_order", "pisa_select", "pisa_attn_fwd_with_sel", "pisa_attn_fwd",
-    "pisa_device_status",
+    "pisa_device_status", "pisa_attn_fwd_with_sel_noalloc",
 )
 
 _p = ctypes.c_void_p
@@ -71,6 +72,8 @@ _lib_first_order = _sig("pisa_block_first_order", _i, _p, _p, _i, _i, _i, _i, _i
 _lib_select = _sig("pisa_select", _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p, _p)
 _lib_fwd_sel = _sig("pisa_attn_fwd_with_sel", _i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i,
                     _p, _p, _p, _p, _i, _p, _z, _p)
+_lib_fwd_sel_noalloc = _sig("pisa_attn_fwd_with_sel_noalloc", _i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i,
+                            _p, _p, _p, _p, _i, _p)
 _lib_fwd = _sig("pisa_attn_fwd", _i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p, _z, _p)
 _lib_device_status = _sig("pisa_device_status", _i, _p, _i)
 
@@ -201,6 +204,20 @@ def attn_fwd_with_sel(q, k, v, block, kbar, vsum, hbar, sel, out=None, workspace
     _check(_lib_fwd_sel(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), b, h, L, d, block,
                         _ptr(kbar), _ptr(vsum), _ptr(hbar), _ptr(sel), int(sel.shape[-1]), _ptr(ws),
                         ws.numel(), _stream(stream)), "pisa_attn_fwd_with_sel")
+    return out
+
+
+def attn_fwd_with_sel_noalloc(q, k, v, block, kbar, vsum, hbar, sel, out=None, stream=None):
+    """attn_fwd_with_sel for callers that cannot allocate device scratch: the
+    library's fixed device array is used instead of a workspace.  Concurrent
+    calls on different streams race on that array."""
+    _need_cuda(q, k, v, kbar, vsum, hbar, sel)
+    b, h, L, d = _qkv_shape(q)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(_lib_fwd_sel_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), b, h, L, d, block,
+                                _ptr(kbar), _ptr(vsum), _ptr(hbar), _ptr(sel), int(sel.shape[-1]),
+                                _stream(stream)), "pisa_attn_fwd_with_sel_noalloc")
     return out
 
 

@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <type_traits>
 
 #include "common.cuh"
@@ -352,6 +353,32 @@ struct FusedOp {
 bool valid_dtype(pisa_dtype dt) { return dt == PISA_BF16 || dt == PISA_FP32; }
 
 }  // namespace
+
+// Scratch of pisa_attn_fwd_with_sel_noalloc: one fixed device array per GPU
+// that loads the library (held until the process exits).  Host code may not
+// use the name as an address: the device address is looked up once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PISA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the scratch array for the current device; the first call
+// on a device resolves it with that device current.
+pisa_status noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PISA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return PISA_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return PISA_OK;
+}
+}  // namespace
 }  // namespace pisa
 
 using namespace pisa;
@@ -455,6 +482,22 @@ pisa_status pisa_attn_fwd_with_sel(const void* q, const void* k, const void* v, 
   if (dtype == PISA_BF16 && (workspace == nullptr || workspace_bytes < fused_ws(s))) return PISA_ERR_WORKSPACE;
   if (workspace != nullptr && !aligned16(workspace)) return PISA_ERR_INVALID_ARG;
   return dispatch<FusedOp>(dtype, d, q, k, v, out, s, kbar, vsum, hbar, sel, k_sel, workspace,
+                           (cudaStream_t)stream);
+}
+
+pisa_status pisa_attn_fwd_with_sel_noalloc(const void* q, const void* k, const void* v, void* out,
+                                           pisa_dtype dtype, int batch, int heads, int L, int d, int block,
+                                           const float* kbar, const float* vsum, const float* hbar,
+                                           const int32_t* sel, int k_sel, void* stream) {
+  const Shape s{batch, heads, L, d, block};
+  if (pisa_status e = check_shape(s)) return e;
+  if (!valid_dtype(dtype)) return PISA_ERR_INVALID_ARG;
+  if (k_sel < 1 || k_sel > s.nb()) return PISA_ERR_INVALID_ARG;
+  if (!all_ok(q, k, v, out, kbar, vsum, hbar) || sel == nullptr) return PISA_ERR_INVALID_ARG;
+  if (fused_ws(s) > PISA_NOALLOC_SCRATCH_BYTES) return PISA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if (pisa_status e = noalloc_scratch(&scratch)) return e;
+  return dispatch<FusedOp>(dtype, d, q, k, v, out, s, kbar, vsum, hbar, sel, k_sel, scratch,
                            (cudaStream_t)stream);
 }
 
