@@ -408,7 +408,7 @@ def main():
     fused_ms = stage_ms["fused"]
     achieved = flops / (fused_ms * 1e-3) / 1e12
     peak = peaks["bf16_sustained"]
-    traffic = stored_traffic("fused", cfg.name)
+    traffic = stored_traffic("fused", f"{cfg.name}:{cfg.heads}")
     roofline = {"kernel": "fused attention (attn_fwd_with_sel)", "bound": "tensor",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "traffic": traffic,
