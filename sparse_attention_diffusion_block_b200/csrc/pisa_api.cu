@@ -197,7 +197,7 @@ pisa_status run_select(const float* qbar, const float* kbar, const float* M, con
   const int nb = s.nb();
   const int R = select_rows(nb);
   if (R < 1) return PISA_ERR_UNSUPPORTED;
-  const size_t smem = ((size_t)R * D + 32 * (D + 4) + R + 64 + (size_t)R * nb) * sizeof(float);
+  const size_t smem = ((size_t)32 * D + 64 * (D + 4) + 32 + 128 + (size_t)R * nb) * sizeof(float);
   if (!set_smem(select_kernel<D>, smem)) return PISA_ERR_CUDA;
   const float scale = 1.0f / sqrtf((float)D);
   select_kernel<D><<<dim3((nb + R - 1) / R, s.BH()), 256, smem, st>>>(qbar, kbar, M, s.L, s.block, nb,

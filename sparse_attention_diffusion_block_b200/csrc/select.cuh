@@ -15,12 +15,14 @@ __device__ __forceinline__ uint32_t orderable_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Grid (ceil(nb / R), BH), 256 threads (8 warps), dynamic smem:
-//   Qb [R][D] fp32, Kc [32][D+4] fp32, keys [R][nb] uint32, qn [R], mj [32], nj [32].
-// Phase 1 computes the R x nb scores with fp32 FMAs (tile of 32 key blocks at a
-// time) and stores their orderable keys; phase 2 runs, per row (one warp per
-// row), an MSB-first bitwise search for the k-th largest key, then writes the
-// selected indices in ascending order.
+// Grid (ceil(nb / R), BH), 256 threads (8 warps), R <= 32, dynamic smem:
+//   Qb [32][D] fp32 (rows >= R zero), Kc [64][D+4] fp32, qn [32], mj [64],
+//   nj [64], keys [R][nb] uint32.
+// Phase 1 computes the R x nb scores with fp32 FMAs, 64 key blocks at a time,
+// each thread a 2 x 4 register tile (rows tr, tr+16; key columns tc + 16c), and
+// stores their orderable keys; phase 2 runs, per row (one warp per row), an
+// MSB-first bitwise search for the k-th largest key, then writes the selected
+// indices in ascending order.
 template <int D>
 __global__ void __launch_bounds__(256)
 select_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
@@ -28,59 +30,77 @@ select_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
               float scale, int32_t* __restrict__ sel) {
   extern __shared__ __align__(16) float sm[];
   constexpr int KS = D + 4;
-  float* Qb = sm;                              // R * D
-  float* Kc = Qb + R * D;                      // 32 * KS
-  float* qn = Kc + 32 * KS;                    // R
-  float* mj = qn + R;                          // 32
-  float* nj = mj + 32;                         // 32
-  uint32_t* keys = reinterpret_cast<uint32_t*>(nj + 32);  // R * nb
+  constexpr int KT = 64;                       // key blocks per tile
+  float* Qb = sm;                              // 32 * D
+  float* Kc = Qb + 32 * D;                     // KT * KS
+  float* qn = Kc + KT * KS;                    // 32
+  float* mj = qn + 32;                         // KT
+  float* nj = mj + KT;                         // KT
+  uint32_t* keys = reinterpret_cast<uint32_t*>(nj + KT);  // R * nb
   const int bh = blockIdx.y;
   const int i0 = blockIdx.x * R;
   const int rows = min(R, nb - i0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  for (int e = threadIdx.x; e < R * D; e += blockDim.x) {
+  for (int e = threadIdx.x; e < 32 * D; e += blockDim.x) {
     const int r = e / D;
     Qb[e] = (r < rows) ? qbar[((size_t)bh * nb + i0 + r) * D + (e % D)] : 0.f;
   }
   __syncthreads();
-  for (int r = warp; r < R; r += 8) {
+  for (int r = warp; r < 32; r += 8) {
     float t = 0.f;
     for (int a = lane; a < D; a += 32) t = fmaf(Qb[r * D + a], Qb[r * D + a], t);
     t = warp_sum(t);
     if (lane == 0) qn[r] = sqrtf(t);
   }
 
-  // Phase 1: scores.  Thread t handles key column c = t % 32 of the tile and
-  // rows r = t / 32, t / 32 + 8, ...
-  for (int j0 = 0; j0 < nb; j0 += 32) {
+  // Phase 1: scores.
+  const int tr = threadIdx.x >> 4, tc = threadIdx.x & 15;
+  for (int j0 = 0; j0 < nb; j0 += KT) {
     __syncthreads();
-    for (int e = threadIdx.x; e < 32 * D; e += blockDim.x) {
-      const int c = e / D, a = e % D;
-      Kc[c * KS + a] = (j0 + c < nb) ? kbar[((size_t)bh * nb + j0 + c) * D + a] : 0.f;
+    for (int e = threadIdx.x; e < KT * (D / 4); e += blockDim.x) {
+      const int c = e / (D / 4), a = (e % (D / 4)) * 4;
+      float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j0 + c < nb) w = *reinterpret_cast<const float4*>(kbar + ((size_t)bh * nb + j0 + c) * D + a);
+      *reinterpret_cast<float4*>(Kc + c * KS + a) = w;
     }
-    if (threadIdx.x < 32) {
+    if (threadIdx.x < KT) {
       const int j = j0 + threadIdx.x;
       mj[threadIdx.x] = (j < nb) ? M[(size_t)bh * nb + j] : 0.f;
       nj[threadIdx.x] = (j < nb) ? (float)min(B, L - j * B) : 1.f;
     }
     __syncthreads();
-    const int c = lane;
-    const int j = j0 + c;
-    if (j < nb) {
-      for (int r = warp; r < rows; r += 8) {
-        float dot = 0.f;
-#pragma unroll 8
-        for (int a = 0; a < D; a += 4) {
-          const float4 x = *reinterpret_cast<const float4*>(Qb + r * D + a);
-          const float4 y = *reinterpret_cast<const float4*>(Kc + c * KS + a);
-          dot = fmaf(x.x, y.x, dot);
-          dot = fmaf(x.y, y.y, dot);
-          dot = fmaf(x.z, y.z, dot);
-          dot = fmaf(x.w, y.w, dot);
-        }
-        const float sc = scale * dot + logf(nj[c] + scale * qn[r] * mj[c]);
-        keys[r * nb + j] = orderable_key(sc);
+    float acc[2][4];
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+#pragma unroll 4
+    for (int a = 0; a < D; a += 4) {
+      const float4 q0 = *reinterpret_cast<const float4*>(Qb + tr * D + a);
+      const float4 q1 = *reinterpret_cast<const float4*>(Qb + (tr + 16) * D + a);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const float4 k = *reinterpret_cast<const float4*>(Kc + (tc + 16 * c) * KS + a);
+        acc[0][c] = fmaf(q0.x, k.x, acc[0][c]);
+        acc[0][c] = fmaf(q0.y, k.y, acc[0][c]);
+        acc[0][c] = fmaf(q0.z, k.z, acc[0][c]);
+        acc[0][c] = fmaf(q0.w, k.w, acc[0][c]);
+        acc[1][c] = fmaf(q1.x, k.x, acc[1][c]);
+        acc[1][c] = fmaf(q1.y, k.y, acc[1][c]);
+        acc[1][c] = fmaf(q1.z, k.z, acc[1][c]);
+        acc[1][c] = fmaf(q1.w, k.w, acc[1][c]);
+      }
+    }
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const int r = tr + 16 * rr;
+      if (r >= rows) continue;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int cl = tc + 16 * c;
+        const int j = j0 + cl;
+        if (j < nb) keys[r * nb + j] = orderable_key(scale * acc[rr][c] + logf(nj[cl] + scale * qn[r] * mj[cl]));
       }
     }
   }
@@ -90,15 +110,51 @@ select_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
   const int C = (nb + 31) / 32;  // contiguous chunk of indices per lane
   for (int r = warp; r < rows; r += 8) {
     const uint32_t* kr = keys + r * nb;
-    uint32_t prefix = 0;
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = prefix | (1u << bit);
-      int cnt = 0;
-      for (int j = lane; j < nb; j += 32) cnt += (kr[j] >= cand);
-      cnt = __reduce_add_sync(0xffffffffu, cnt);
-      if (cnt >= kk) prefix = cand;
+    uint32_t thr;  // k-th largest key
+    if (nb <= 1024) {
+      // keys in registers (j = lane + 32 m; a 0 key stands for "no block" and
+      // is never counted since every candidate is >= 1)
+      uint32_t kv[32];
+      uint32_t mx = 0u, mn = 0xffffffffu;
+#pragma unroll
+      for (int m = 0; m < 32; ++m) {
+        const int j = lane + 32 * m;
+        kv[m] = (j < nb) ? kr[j] : 0u;
+        if (j < nb) {
+          mx = max(mx, kv[m]);
+          mn = min(mn, kv[m]);
+        }
+      }
+      mx = __reduce_max_sync(0xffffffffu, mx);
+      mn = __reduce_min_sync(0xffffffffu, mn);
+      // the k-th largest lies in [mn, mx], so it shares their common high bits
+      const uint32_t diff = mx ^ mn;
+      if (diff == 0u) {
+        thr = mx;
+      } else {
+        const int top = 31 - __clz(diff);
+        uint32_t prefix = (top == 31) ? 0u : (mx & ~((2u << top) - 1u));
+        for (int bit = top; bit >= 0; --bit) {
+          const uint32_t cand = prefix | (1u << bit);
+          int cnt = 0;
+#pragma unroll
+          for (int m = 0; m < 32; ++m) cnt += (kv[m] >= cand);
+          cnt = __reduce_add_sync(0xffffffffu, cnt);
+          if (cnt >= kk) prefix = cand;
+        }
+        thr = prefix;
+      }
+    } else {
+      uint32_t prefix = 0;
+      for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cand = prefix | (1u << bit);
+        int cnt = 0;
+        for (int j = lane; j < nb; j += 32) cnt += (kr[j] >= cand);
+        cnt = __reduce_add_sync(0xffffffffu, cnt);
+        if (cnt >= kk) prefix = cand;
+      }
+      thr = prefix;
     }
-    const uint32_t thr = prefix;  // k-th largest key
     const int jb = lane * C, je = min(nb, jb + C);
     int n_gt = 0, n_eq = 0;
     for (int j = jb; j < je; ++j) {
