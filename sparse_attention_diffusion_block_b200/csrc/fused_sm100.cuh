@@ -25,7 +25,10 @@
 // Work list of a pair: the exact KV blocks of each tile (for 64-token blocks a
 // 128-row tile spans two query blocks: the union, with per-row-group bits),
 // blocks selected by both tiles first and in the same order, so those K/V
-// tiles are loaded once and feed both; then the centroid tiles (128 key
+// tiles are loaded once and feed both.  Every step covers 128 keys: one
+// 128-token block, or two consecutive 64-token entries stacked in one ring
+// slot (each 64-column half of S masked by its own entry), so the MMAs are
+// always 128 x 128.  Then the centroid tiles (128 key
 // centroids each, shared by both tiles, masked per tile); fp32 statistics
 // enter as bf16 hi + lo MMA pairs.  q_t Hbar (Hbar as hi + lo) runs last into
 // the tile's S columns.
@@ -240,34 +243,54 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             }
           }
         }
-        L_[0] = nA;
-        L_[1] = nB;
-        L_[2] = nC;
+        // header: steps of A, B and shared steps (a step = 128 keys: one 128-token
+        // block, or two consecutive list entries of 64 tokens), then the entry counts
+        L_[0] = (nA + G - 1) / G;
+        L_[1] = (nB + G - 1) / G;
+        L_[2] = nC / G;
         L_[3] = existsB;
         L_[4] = bh;
         L_[5] = tA;
+        L_[6] = nA;
+        L_[7] = nB;
         mbar_arrive(&list_full[slot]);
 
-        const PairPlan pl{nA, nB, nC, existsB, n_cent};
-        auto load = [&](const CUtensorMap* map, int row, int rows) -> bool {
+        const PairPlan pl{(nA + G - 1) / G, (nB + G - 1) / G, nC / G, existsB, n_cent};
+        // one ring item: `rows` rows at `row`, and when row2 >= 0 another `rows`
+        // rows at row2 stacked below them (a 2 x 64-row step)
+        auto load = [&](const CUtensorMap* map, int row, int rows, int row2) -> bool {
           const int s = it % NS;
           if (!mbar_wait(&empty[s], ((it / NS) & 1) ^ 1, abort)) return false;
-          mbar_expect_tx(&full[s], rows * D * 2);
+          const int tile_rows = row2 >= 0 ? 2 * rows : rows;
+          mbar_expect_tx(&full[s], tile_rows * D * 2);
 #pragma unroll
-          for (int cb = 0; cb < CB; ++cb)
-            tma_load_3d(sRing + s * SLOT + cb * rows * 128, map, &full[s], cb * 64, row, bh);
+          for (int cb = 0; cb < CB; ++cb) {
+            uint8_t* dst = sRing + s * SLOT + cb * tile_rows * 128;
+            tma_load_3d(dst, map, &full[s], cb * 64, row, bh);
+            if (row2 >= 0) tma_load_3d(dst + rows * 128, map, &full[s], cb * 64, row2, bh);
+          }
           ++it;
           return true;
         };
+        // exact step u of tile x: entries G u .. G u + G - 1; a missing second
+        // 64-token entry repeats the first (in bounds; its columns are masked)
+        auto exact_item = [&](const CUtensorMap* map, int x, int u) -> bool {
+          const int* e = x ? eB : eA;
+          const int n = x ? nB : nA;
+          const int j1 = e[G * u] & 0xFFFFFF;
+          if (G == 1) return load(map, j1 * KB, KB, -1);
+          const int j2 = (G * u + 1 < n) ? (e[G * u + 1] & 0xFFFFFF) : j1;
+          return load(map, j1 * KB, KB, j2 * KB);
+        };
         auto loadK = [&](int x, int u) -> bool {
-          if (!pl.centroid(u)) return load(&tmK, ((x ? eB : eA)[u] & 0xFFFFFF) * KB, KB);
+          if (!pl.centroid(u)) return exact_item(&tmK, x, u);
           const int c = u - pl.U();
-          return load(&tmKc, c * 128, 128) && load(&tmKc, a.nbp + c * 128, 128);
+          return load(&tmKc, c * 128, 128, -1) && load(&tmKc, a.nbp + c * 128, 128, -1);
         };
         auto loadV = [&](int x, int u) -> bool {
-          if (!pl.centroid(u)) return load(&tmV, ((x ? eB : eA)[u] & 0xFFFFFF) * KB, KB);
+          if (!pl.centroid(u)) return exact_item(&tmV, x, u);
           const int c = u - pl.U();
-          return load(&tmVc, c * 128, 128) && load(&tmVc, a.nbp + c * 128, 128);
+          return load(&tmVc, c * 128, 128, -1) && load(&tmVc, a.nbp + c * 128, 128, -1);
         };
         for (int x = 0; ok && x < 1 + existsB; ++x) {
           ok = mbar_wait(&q_empty[x], (qloads[x] & 1) ^ 1, abort);
@@ -287,7 +310,7 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           if (ok && pl.activeB(u) && !pl.shared(u)) ok = loadV(1, u);
           if (ok && u + 1 < T && pl.activeB(u + 1) && !pl.shared(u + 1)) ok = loadK(1, u + 1);
         }
-        if (ok) ok = load(&tmH, 0, D) && load(&tmH, D, D);
+        if (ok) ok = load(&tmH, 0, D, -1) && load(&tmH, D, D, -1);
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     }
@@ -299,8 +322,7 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
    } else if (warp == 9) {
     // ================================================================ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(128, KB, false, false);
-      constexpr uint32_t idC = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idC = idesc_bf16(128, 128, false, false);  // every step is 128 keys
       constexpr uint32_t idH = idesc_bf16(128, D, false, false);
       constexpr uint32_t idO = idesc_bf16(128, D, false, true);
       const uint32_t ring = smem_u32(sRing);
@@ -350,7 +372,7 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             }
           }
           if (!pl.centroid(u)) {
-            for (int kk = 0; kk < D / 16; ++kk) mma_ss(sc, qdesc(x, kk), kdesc(ks[0], KB, kk), idS, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) mma_ss(sc, qdesc(x, kk), kdesc(ks[0], 128, kk), idC, kk > 0 ? 1u : 0u);
           } else {
             for (int kk = 0; kk < D / 16; ++kk) mma_ss(sc, qdesc(x, kk), kdesc(ks[0], 128, kk), idC, kk > 0 ? 1u : 0u);
             for (int kk = 0; kk < D / 16; ++kk) mma_ss(sc, qdesc(x, kk), kdesc(ks[1], 128, kk), idC, 1u);
@@ -377,8 +399,8 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             }
           }
           if (!pl.centroid(u)) {
-            for (int kk = 0; kk < KB / 16; ++kk)
-              mma_ts(oc, pa + kk * 8, vdesc(vs[0], KB, kk), idO, (!first_pv[x] || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ts(oc, pa + kk * 8, vdesc(vs[0], 128, kk), idO, (!first_pv[x] || kk > 0) ? 1u : 0u);
           } else {
             for (int kk = 0; kk < 8; ++kk)
               mma_ts(oc, pa + kk * 8, vdesc(vs[0], 128, kk), idO, (!first_pv[x] || kk > 0) ? 1u : 0u);
@@ -453,6 +475,7 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const int bh = L_[4];
       const int qtile = L_[5] + x;
       const int* ent = L_ + 8 + x * G * a.kk;
+      const int n_ent = L_[6 + x];
       const uint32_t* msk = reinterpret_cast<const uint32_t*>(L_ + 8 + 2 * G * a.kk) + x * G * words + g * words;
       if (x == 0 || pl.existsB) {
         const int qrow = qtile * QT + row;
@@ -469,36 +492,40 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           fence_after_sync();
           const bool exact = !pl.centroid(u);
           float tmax = -INFINITY, x_tail = -INFINITY;
-          int ncols = 128;
+          tmem_ld32(sbase, s);
+          tmem_ld32(sbase + 32, s + 32);
+          tmem_ld32(sbase + 64, s + 64);
+          tmem_ld32(sbase + 96, s + 96);
+          tmem_wait_ld();
           if (exact) {
-            ncols = KB;
-            tmem_ld32(sbase, s);
-            tmem_ld32(sbase + 32, s + 32);
-            if (KB == 128) {
-              tmem_ld32(sbase + 64, s + 64);
-              tmem_ld32(sbase + 96, s + 96);
-            }
-            tmem_wait_ld();
-            const int e = ent[u];
-            const int j = e & 0xFFFFFF;
-            const int nvalid = ((e >> (24 + g)) & 1) ? min(KB, a.L - j * KB) : 0;
-            if (__all_sync(0xffffffffu, nvalid == KB)) {
+            // column half h (of KB columns) holds list entry G u + h; the keys of
+            // that block this row may use: all of its tokens if the row's query
+            // block selected it, none otherwise (or when the entry is absent)
+            int nvalid[G];
 #pragma unroll
-              for (int c = 0; c < KB; ++c) tmax = fmaxf(tmax, __uint_as_float(s[c]));
+            for (int h = 0; h < G; ++h) {
+              nvalid[h] = 0;
+              if (G * u + h < n_ent) {
+                const int e = ent[G * u + h];
+                const int j = e & 0xFFFFFF;
+                if ((e >> (24 + g)) & 1) nvalid[h] = min(KB, a.L - j * KB);
+              }
+            }
+            bool whole = true;
+#pragma unroll
+            for (int h = 0; h < G; ++h) whole = whole && nvalid[h] == KB;
+            if (__all_sync(0xffffffffu, whole)) {
+#pragma unroll
+              for (int c = 0; c < 128; ++c) tmax = fmaxf(tmax, __uint_as_float(s[c]));
             } else {
 #pragma unroll
-              for (int c = 0; c < KB; ++c) {
-                const float v = c < nvalid ? __uint_as_float(s[c]) : -INFINITY;
+              for (int c = 0; c < 128; ++c) {
+                const float v = (c % KB) < nvalid[c / KB] ? __uint_as_float(s[c]) : -INFINITY;
                 s[c] = __float_as_uint(v);
                 tmax = fmaxf(tmax, v);
               }
             }
           } else {
-            tmem_ld32(sbase, s);
-            tmem_ld32(sbase + 32, s + 32);
-            tmem_ld32(sbase + 64, s + 64);
-            tmem_ld32(sbase + 96, s + 96);
-            tmem_wait_ld();
             const int c0 = (u - pl.U()) * 128;
             const uint32_t* mw = msk + c0 / 32;
 #pragma unroll
@@ -545,13 +572,11 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           uint64_t acc = 0;
 #pragma unroll
           for (int c = 0; c < 128; c += 2) {
-            if (c < ncols) {
-              const uint64_t t = ffma2(f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), c2x2, nmu);
-              const float p0 = ex2(f2_lo(t));
-              const float p1 = ex2(f2_hi(t));
-              acc = fadd2(acc, f2_pack(p0, p1));
-              s[c >> 1] = pack_bf16x2(p0, p1);
-            }
+            const uint64_t t = ffma2(f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), c2x2, nmu);
+            const float p0 = ex2(f2_lo(t));
+            const float p1 = ex2(f2_hi(t));
+            acc = fadd2(acc, f2_pack(p0, p1));
+            s[c >> 1] = pack_bf16x2(p0, p1);
           }
           const float sum = f2_lo(acc) + f2_hi(acc);
           if (exact) {
@@ -562,7 +587,7 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             if (x_tail != -INFINITY) l += (float)(n_tail - a.block) * ex2(x_tail * c2 - mu);
           }
           tmem_st32(sbase, s);
-          if (ncols == 128) tmem_st32(sbase + 32, s + 32);
+          tmem_st32(sbase + 32, s + 32);
           tmem_wait_st();
           fence_before_sync();
           mbar_arrive(&p_full[x]);
