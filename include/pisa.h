@@ -146,6 +146,49 @@ pisa_status pisa_attn_fwd(const void* q, const void* k, const void* v, void* out
                           float keep_ratio, void* workspace, size_t workspace_bytes,
                           void* stream);
 
+/* Device workspace bytes pisa_attn_fwd_host needs when it works through the
+ * (batch, head) slices `chunk` at a time: the scratch of pisa_attn_fwd for
+ * one chunk plus two device staging copies of a chunk's q, k, v and out.
+ * Returns 0 for unsupported shapes or dtype, k outside [1, nb] or chunk < 1. */
+size_t pisa_host_workspace_size(pisa_dtype dtype, int batch, int heads, int L, int d, int block, int k,
+                                int chunk);
+
+/* pisa_attn_fwd for tensors that live in HOST memory.  The pages describe the
+ * forward only; this entry point is an interface convenience for callers whose
+ * q, k, v and out are host-resident, and it overlaps the PCIe copies with the
+ * compute instead of running copy, compute, copy back to back.
+ *   q_host, k_host, v_host, out_host: [batch, heads, L, d] in host memory, the
+ *   element type of `dtype`.  workspace: device memory owned by the caller,
+ *   16-byte aligned, >= pisa_host_workspace_size(dtype, ..., k, chunk) with
+ *   k = pisa_keep_count(L, block, keep_ratio).
+ *   The batch*heads slices go through in chunks of `chunk` consecutive slices
+ *   (the last chunk may be shorter).  For each chunk: the inputs are copied in
+ *   on an internal copy stream, the whole forward (stats, covariance norm,
+ *   routing, fused attention) runs on `stream`, and the output is copied back
+ *   on a second internal copy stream.  Two staging buffers let the next
+ *   chunk's input copy and the previous chunk's output copy run while a chunk
+ *   computes.
+ *   - Asynchronous: returns once everything is enqueued; `stream` reaches the
+ *     end of the last output copy only when all copies and kernels are done.
+ *     The host buffers must stay valid and untouched until then.
+ *   - Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister)
+ *     for the copies to overlap; pageable memory works but copies stall the
+ *     host.
+ *   - Each slice is computed by the same kernels as in pisa_attn_fwd.  The
+ *     fixed-order partial sums behind Hbar are grouped by the number of slices
+ *     per launch, so results can differ from one whole-batch pisa_attn_fwd
+ *     call in the last bits unless chunk >= batch*heads.
+ *   - The library keeps, per device, two non-blocking copy streams and a few
+ *     events, created on the first call on that device and kept until exit.
+ *     Calls on one device are enqueued under a lock and share those streams.
+ *   - Arguments are validated before any CUDA call: null pointers or chunk < 1
+ *     give PISA_ERR_INVALID_ARG, a missing or small workspace
+ *     PISA_ERR_WORKSPACE; a failing copy or launch gives PISA_ERR_CUDA. */
+pisa_status pisa_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
+                               void* out_host, pisa_dtype dtype, int batch, int heads, int L,
+                               int d, int block, float keep_ratio, int chunk, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
 /* Size in bytes of the fixed device scratch array used by
  * pisa_attn_fwd_with_sel_noalloc (32 MiB). */
 #define PISA_NOALLOC_SCRATCH_BYTES (32ull * 1024ull * 1024ull)

@@ -7,8 +7,8 @@ loudly when the library has not been built.
 
 Entry points mirror the C names (without the ``pisa_`` prefix):
 block_stats, cov_norm, block_first_order, select, attn_fwd_with_sel, attn_fwd,
-attn_fwd_with_sel_noalloc, keep_count, workspace_size, stats_workspace_size, fused_workspace_size,
-device_status, status_string.
+attn_fwd_host, attn_fwd_with_sel_noalloc, keep_count, workspace_size, stats_workspace_size,
+fused_workspace_size, host_workspace_size, device_status, status_string.
 """
 
 from __future__ import annotations
@@ -44,7 +44,8 @@ EXPORTS = (
     "pisa_status_string", "pisa_keep_count", "pisa_stats_workspace_size",
     "pisa_fused_workspace_size", "pisa_workspace_size", "pisa_block_stats", "pisa_cov_norm",
     "pisa_block_first_order", "pisa_select", "pisa_attn_fwd_with_sel", "pisa_attn_fwd",
-    "pisa_device_status", "pisa_attn_fwd_with_sel_noalloc",
+    "pisa_device_status", "pisa_attn_fwd_with_sel_noalloc", "pisa_host_workspace_size",
+    "pisa_attn_fwd_host",
 )
 
 _p = ctypes.c_void_p
@@ -76,6 +77,8 @@ _lib_fwd_sel_noalloc = _sig("pisa_attn_fwd_with_sel_noalloc", _i, _p, _p, _p, _p
                             _p, _p, _p, _p, _i, _p)
 _lib_fwd = _sig("pisa_attn_fwd", _i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p, _z, _p)
 _lib_device_status = _sig("pisa_device_status", _i, _p, _i)
+_lib_host_ws = _sig("pisa_host_workspace_size", _z, _i, _i, _i, _i, _i, _i, _i, _i)
+_lib_fwd_host = _sig("pisa_attn_fwd_host", _i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _i, _p, _z, _p)
 
 
 class PisaError(RuntimeError):
@@ -142,6 +145,11 @@ def fused_workspace_size(batch, heads, L, d, block) -> int:
 
 def workspace_size(batch, heads, L, d, block, k) -> int:
     return int(_lib_ws(batch, heads, L, d, block, k))
+
+
+def host_workspace_size(dtype: torch.dtype, batch, heads, L, d, block, k, chunk) -> int:
+    code = PISA_BF16 if dtype == torch.bfloat16 else PISA_FP32 if dtype == torch.float32 else -1
+    return int(_lib_host_ws(code, batch, heads, L, d, block, k, chunk))
 
 
 def _workspace(nbytes: int, device, given: Optional[torch.Tensor]):
@@ -231,6 +239,31 @@ def attn_fwd(q, k, v, block, keep_ratio, out=None, workspace=None, stream=None):
     ws = _workspace(workspace_size(b, h, L, d, block, kk), q.device, workspace)
     _check(_lib_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), b, h, L, d, block,
                     float(keep_ratio), _ptr(ws), ws.numel(), _stream(stream)), "pisa_attn_fwd")
+    return out
+
+
+def attn_fwd_host(q, k, v, block, keep_ratio, out=None, chunk=4, workspace=None, stream=None,
+                  device=None):
+    """PISA forward on HOST tensors [b,h,L,d]: the library copies chunks of
+    ``chunk`` (batch, head) slices in, runs the forward and copies the result
+    back, overlapping copies with compute.  Pin the host tensors
+    (``tensor.pin_memory()``) for the copies to overlap.  Asynchronous on
+    ``stream``: synchronise it before reading ``out``.  ``workspace`` is a
+    device byte tensor of at least host_workspace_size(...) bytes."""
+    for t in (q, k, v):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous host tensors")
+    b, h, L, d = _qkv_shape(q)
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=q.is_pinned())
+    if out.is_cuda or not out.is_contiguous() or out.shape != q.shape or out.dtype != q.dtype:
+        raise ValueError("out must be a contiguous host tensor shaped and typed like q")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    kk = keep_count(L, block, keep_ratio)
+    ws = _workspace(host_workspace_size(q.dtype, b, h, L, d, block, kk, chunk), dev, workspace)
+    _check(_lib_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), b, h, L, d, block,
+                         float(keep_ratio), int(chunk), _ptr(ws), ws.numel(), _stream(stream)),
+           "pisa_attn_fwd_host")
     return out
 
 

@@ -378,6 +378,129 @@ pisa_status noalloc_scratch(void** out) {
   *out = g_noalloc_addr[dev];
   return PISA_OK;
 }
+// The whole forward on device tensors of shape s (arguments already checked).
+pisa_status forward_device(const void* q, const void* k, const void* v, void* out, pisa_dtype dtype,
+                           const Shape& s, int kk, void* workspace, cudaStream_t st) {
+  const Carve c = carve(s, kk, static_cast<char*>(workspace));
+  const int d = s.d;
+  pisa_status e = dispatch<StatsOp>(dtype, d, q, k, v, s, c.qbar, c.kbar, c.vsum, c.hbar, (float*)c.stats, st);
+  if (e) return e;
+  e = dispatch<CovNormOp>(dtype, d, k, v, s, (const float*)c.kbar, (const float*)c.vsum,
+                          (const float*)c.hbar, c.M, st);
+  if (e) return e;
+  e = d == 128 ? run_select<128>(c.qbar, c.kbar, c.M, s, kk, c.sel, st)
+               : run_select<64>(c.qbar, c.kbar, c.M, s, kk, c.sel, st);
+  if (e) return e;
+  return dispatch<FusedOp>(dtype, d, q, k, v, out, s, (const float*)c.kbar, (const float*)c.vsum,
+                           (const float*)c.hbar, (const int32_t*)c.sel, kk, c.fused, st);
+}
+
+// ------------------------------------------------------------------ host-buffer forward
+//
+// Device workspace of pisa_attn_fwd_host: [forward scratch of one chunk]
+// [slot 0: q, k, v, out of one chunk][slot 1: the same], each piece 256-byte
+// aligned.  Sized for the widest element type (fp32) so one size query covers
+// both dtypes.
+struct HostPlan {
+  int chunk;     // slices per chunk (clamped to batch*heads)
+  size_t fwd;    // forward scratch: the larger of a full chunk's and the last chunk's
+  size_t piece;  // one staged tensor of a full chunk
+  size_t total() const { return align_up(fwd) + 8 * piece; }
+  size_t slot_stride() const { return 4 * piece; }
+};
+
+HostPlan host_plan(const Shape& s, int kk, int chunk, pisa_dtype dtype) {
+  HostPlan hp{};
+  hp.chunk = chunk < s.BH() ? chunk : s.BH();
+  const size_t es = dtype == PISA_BF16 ? 2 : 4;
+  hp.piece = align_up((size_t)hp.chunk * s.L * s.d * es);
+  // the stats scratch is not monotonic in the slice count, so size both chunk shapes that occur
+  hp.fwd = carve(Shape{1, hp.chunk, s.L, s.d, s.block}, kk, nullptr).total;
+  const int tail = s.BH() % hp.chunk;
+  if (tail) {
+    const size_t t = carve(Shape{1, tail, s.L, s.d, s.block}, kk, nullptr).total;
+    if (t > hp.fwd) hp.fwd = t;
+  }
+  return hp;
+}
+
+// Per-device copy streams and events of the host-buffer forward, created on
+// the first call on that device and kept until the process exits.
+struct HostPipe {
+  bool ready = false;
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, fin = nullptr;
+  cudaEvent_t in_done[2] = {}, comp_done[2] = {}, out_done[2] = {};
+};
+std::mutex g_pipe_mutex;
+HostPipe g_pipe[kMaxDevices];
+
+pisa_status host_pipe(HostPipe** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PISA_ERR_CUDA;
+  HostPipe& p = g_pipe[dev];
+  if (!p.ready) {
+    const unsigned ev = cudaEventDisableTiming;
+    if (cudaStreamCreateWithFlags(&p.in, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&p.out, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&p.start, ev) != cudaSuccess || cudaEventCreateWithFlags(&p.fin, ev) != cudaSuccess)
+      return PISA_ERR_CUDA;
+    for (int i = 0; i < 2; ++i)
+      if (cudaEventCreateWithFlags(&p.in_done[i], ev) != cudaSuccess ||
+          cudaEventCreateWithFlags(&p.comp_done[i], ev) != cudaSuccess ||
+          cudaEventCreateWithFlags(&p.out_done[i], ev) != cudaSuccess)
+        return PISA_ERR_CUDA;
+    p.ready = true;
+  }
+  *out = &p;
+  return PISA_OK;
+}
+
+pisa_status forward_host(const void* qh, const void* kh, const void* vh, void* oh, pisa_dtype dtype,
+                         const Shape& s, int kk, const HostPlan& hp, char* ws, cudaStream_t st) {
+  std::lock_guard<std::mutex> lock(g_pipe_mutex);
+  HostPipe* p = nullptr;
+  if (pisa_status e = host_pipe(&p)) return e;
+  const size_t es = dtype == PISA_BF16 ? 2 : 4;
+  const size_t slice = (size_t)s.L * s.d * es;
+  char* fwd_ws = ws;
+  char* slots = ws + align_up(hp.fwd);
+  auto dev = [&](int slot, int t) { return slots + slot * hp.slot_stride() + t * hp.piece; };
+  const char* src[3] = {static_cast<const char*>(qh), static_cast<const char*>(kh), static_cast<const char*>(vh)};
+  char* dst = static_cast<char*>(oh);
+  // copies start after the work already queued on the caller's stream (which
+  // may still be using the workspace)
+  if (cudaEventRecord(p->start, st) != cudaSuccess || cudaStreamWaitEvent(p->in, p->start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(p->out, p->start, 0) != cudaSuccess)
+    return PISA_ERR_CUDA;
+  const int BH = s.BH();
+  for (int c = 0, first = 0; first < BH; ++c, first += hp.chunk) {
+    const int n = BH - first < hp.chunk ? BH - first : hp.chunk;
+    const int sl = c & 1;
+    const size_t off = (size_t)first * slice, bytes = (size_t)n * slice;
+    // inputs of this slot are free once the forward two chunks back has run
+    if (c >= 2 && cudaStreamWaitEvent(p->in, p->comp_done[sl], 0) != cudaSuccess) return PISA_ERR_CUDA;
+    for (int t = 0; t < 3; ++t)
+      if (cudaMemcpyAsync(dev(sl, t), src[t] + off, bytes, cudaMemcpyHostToDevice, p->in) != cudaSuccess)
+        return PISA_ERR_CUDA;
+    if (cudaEventRecord(p->in_done[sl], p->in) != cudaSuccess) return PISA_ERR_CUDA;
+    // the forward needs this chunk's inputs and an output slot already copied out
+    if (cudaStreamWaitEvent(st, p->in_done[sl], 0) != cudaSuccess) return PISA_ERR_CUDA;
+    if (c >= 2 && cudaStreamWaitEvent(st, p->out_done[sl], 0) != cudaSuccess) return PISA_ERR_CUDA;
+    const Shape cs{1, n, s.L, s.d, s.block};
+    if (pisa_status e = forward_device(dev(sl, 0), dev(sl, 1), dev(sl, 2), dev(sl, 3), dtype, cs, kk, fwd_ws, st))
+      return e;
+    if (cudaEventRecord(p->comp_done[sl], st) != cudaSuccess) return PISA_ERR_CUDA;
+    if (cudaStreamWaitEvent(p->out, p->comp_done[sl], 0) != cudaSuccess ||
+        cudaMemcpyAsync(dst + off, dev(sl, 3), bytes, cudaMemcpyDeviceToHost, p->out) != cudaSuccess ||
+        cudaEventRecord(p->out_done[sl], p->out) != cudaSuccess)
+      return PISA_ERR_CUDA;
+  }
+  // the caller's stream completes after the last output copy
+  if (cudaEventRecord(p->fin, p->out) != cudaSuccess || cudaStreamWaitEvent(st, p->fin, 0) != cudaSuccess)
+    return PISA_ERR_CUDA;
+  return PISA_OK;
+}
 }  // namespace
 }  // namespace pisa
 
@@ -513,18 +636,32 @@ pisa_status pisa_attn_fwd(const void* q, const void* k, const void* v, void* out
   const Carve need = carve(s, kk, nullptr);
   if (workspace == nullptr || workspace_bytes < need.total) return PISA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return PISA_ERR_INVALID_ARG;
-  const Carve c = carve(s, kk, static_cast<char*>(workspace));
-  cudaStream_t st = (cudaStream_t)stream;
-  pisa_status e = dispatch<StatsOp>(dtype, d, q, k, v, s, c.qbar, c.kbar, c.vsum, c.hbar, (float*)c.stats, st);
-  if (e) return e;
-  e = dispatch<CovNormOp>(dtype, d, k, v, s, (const float*)c.kbar, (const float*)c.vsum,
-                          (const float*)c.hbar, c.M, st);
-  if (e) return e;
-  e = d == 128 ? run_select<128>(c.qbar, c.kbar, c.M, s, kk, c.sel, st)
-               : run_select<64>(c.qbar, c.kbar, c.M, s, kk, c.sel, st);
-  if (e) return e;
-  return dispatch<FusedOp>(dtype, d, q, k, v, out, s, (const float*)c.kbar, (const float*)c.vsum,
-                           (const float*)c.hbar, (const int32_t*)c.sel, kk, c.fused, st);
+  return forward_device(q, k, v, out, dtype, s, kk, workspace, (cudaStream_t)stream);
+}
+
+size_t pisa_host_workspace_size(pisa_dtype dtype, int batch, int heads, int L, int d, int block, int k,
+                                int chunk) {
+  const Shape s{batch, heads, L, d, block};
+  if (check_shape(s) != PISA_OK || !valid_dtype(dtype) || k < 1 || k > s.nb() || chunk < 1) return 0;
+  return host_plan(s, k, chunk, dtype).total();
+}
+
+pisa_status pisa_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* out_host,
+                               pisa_dtype dtype, int batch, int heads, int L, int d, int block,
+                               float keep_ratio, int chunk, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  const Shape s{batch, heads, L, d, block};
+  if (pisa_status e = check_shape(s)) return e;
+  if (!valid_dtype(dtype)) return PISA_ERR_INVALID_ARG;
+  const int kk = pisa_keep_count(L, block, keep_ratio);
+  if (kk < 1 || chunk < 1) return PISA_ERR_INVALID_ARG;
+  if (q_host == nullptr || k_host == nullptr || v_host == nullptr || out_host == nullptr)
+    return PISA_ERR_INVALID_ARG;
+  const HostPlan hp = host_plan(s, kk, chunk, dtype);
+  if (workspace == nullptr || workspace_bytes < hp.total()) return PISA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return PISA_ERR_INVALID_ARG;
+  return forward_host(q_host, k_host, v_host, out_host, dtype, s, kk, hp, static_cast<char*>(workspace),
+                      (cudaStream_t)stream);
 }
 
 pisa_status pisa_device_status(void* stream, int reset) {

@@ -98,3 +98,45 @@ def test_stage_entry_points_validate(lib):
     assert raw.pisa_attn_fwd_with_sel(FAKE, FAKE, FAKE, FAKE, 0, 1, 1, 1000, 128, 128, FAKE, FAKE, FAKE,
                                       FAKE, 0, FAKE, ctypes.c_size_t(1 << 30), None) == \
         lib.PISA_ERR_INVALID_ARG
+
+
+def test_host_workspace_size(lib):
+    import torch
+    kk = 60
+    full = lib.host_workspace_size(torch.bfloat16, 1, 40, 75600, 128, 128, kk, 8)
+    assert full > 0
+    assert lib.host_workspace_size(torch.float32, 1, 40, 75600, 128, 128, kk, 8) > full
+    assert lib.host_workspace_size(torch.bfloat16, 1, 40, 75600, 128, 128, kk, 0) == 0   # chunk < 1
+    assert lib.host_workspace_size(torch.float16, 1, 40, 75600, 128, 128, kk, 8) == 0    # bad dtype
+    assert lib.host_workspace_size(torch.bfloat16, 1, 40, 75600, 96, 128, kk, 8) == 0    # d = 96
+    # the scratch of the forward is not monotonic in the slice count: a short last
+    # chunk (7 slices) can need more than a full one (8); the size covers both
+    for tail in (7, 8):
+        assert full > lib.workspace_size(1, tail, 75600, 128, 128, kk)
+    assert lib.workspace_size(1, 7, 75600, 128, 128, kk) > lib.workspace_size(1, 8, 75600, 128, 128, kk)
+    # a chunk larger than the slice count is clamped to it
+    assert lib.host_workspace_size(torch.bfloat16, 1, 3, 1000, 128, 128, 2, 64) == \
+        lib.host_workspace_size(torch.bfloat16, 1, 3, 1000, 128, 128, 2, 3)
+
+
+def test_host_entry_point_validates_before_any_cuda_call(lib):
+    raw = lib.raw_lib()
+    f = raw.pisa_attn_fwd_host
+    ok = [FAKE, FAKE, FAKE, FAKE, 0, 1, 2, 1000, 128, 128, ctypes.c_float(0.25), 2, FAKE,
+          ctypes.c_size_t(1 << 40), None]
+
+    def call(**over):
+        a = list(ok)
+        for i, val in over.items():
+            a[int(i[1:])] = val
+        return f(*a)
+
+    assert call(a1=None) == lib.PISA_ERR_INVALID_ARG            # null k_host
+    assert call(a3=None) == lib.PISA_ERR_INVALID_ARG            # null out_host
+    assert call(a11=0) == lib.PISA_ERR_INVALID_ARG              # chunk = 0
+    assert call(a8=80) == lib.PISA_ERR_UNSUPPORTED              # d = 80
+    assert call(a4=3) == lib.PISA_ERR_INVALID_ARG               # bad dtype
+    assert call(a10=ctypes.c_float(0.0)) == lib.PISA_ERR_INVALID_ARG
+    assert call(a12=None) == lib.PISA_ERR_WORKSPACE
+    assert call(a13=ctypes.c_size_t(4096)) == lib.PISA_ERR_WORKSPACE
+    assert call(a12=MISALIGNED) == lib.PISA_ERR_INVALID_ARG
