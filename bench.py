@@ -231,6 +231,120 @@ def run_reference(args, cfg, kk):
 # ------------------------------------------------------------------ GPU path
 
 
+def dense_reference(pisa, cfg, qd, kd, vd, stats, fused_ms, forward_ms, reps=3):
+    """Dense-attention context on the same inputs: this library's fused kernel
+    with every block selected (U_i empty, so the result is exact softmax
+    attention) and torch's scaled_dot_product_attention.  Each is timed with
+    CUDA events over ``reps`` calls after one warm-up call."""
+    import torch
+    b, h, L, d, B, nb = cfg.batch, cfg.heads, cfg.L, cfg.d, cfg.block, cfg.nb
+    dense_flops = 4.0 * L * L * d * b * h
+    out = {"flops": dense_flops}
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            fn()
+        z.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(z) / reps
+
+    sel_all = torch.arange(nb, dtype=torch.int32, device=qd.device).expand(b, h, nb, nb).contiguous()
+    o = torch.empty_like(qd)
+    ws = torch.empty(max(pisa.fused_workspace_size(b, h, L, d, B), 16), dtype=torch.uint8, device=qd.device)
+    ms = timed(lambda: pisa.attn_fwd_with_sel(qd, kd, vd, B, stats[1], stats[2], stats[3], sel_all, out=o,
+                                              workspace=ws))
+    out["pisa_every_block"] = {"ms": ms, "TFLOP/s": dense_flops / (ms * 1e-3) / 1e12}
+    del sel_all, ws
+    try:
+        from torch.nn.functional import scaled_dot_product_attention as sdpa
+        ms = timed(lambda: sdpa(qd, kd, vd))
+        out["torch_sdpa"] = {"ms": ms, "TFLOP/s": dense_flops / (ms * 1e-3) / 1e12}
+        out["pisa_forward_speedup_vs_sdpa"] = ms / forward_ms
+        out["pisa_fused_speedup_vs_sdpa"] = ms / fused_ms
+    except Exception as e:  # noqa: BLE001  (context only: report and go on)
+        out["torch_sdpa"] = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
+    del o
+    torch.cuda.empty_cache()
+    return out
+
+
+SWEEP_GRIDS = {4096: (4, 32, 32), 8192: (8, 32, 32), 16384: (16, 32, 32), 32768: (32, 32, 32)}
+SWEEP_KEEP = (0.05, 0.1, 0.25, 0.5)
+
+
+def run_sweep(args):
+    """Sequence-length x density sweep (4K-32K tokens, the axes of the pages'
+    kernel comparison): 24 heads, d=128, block 128, the video-like generator
+    on a frames x 32 x 32 grid.  For each length: torch SDPA and this
+    library's fused kernel with every block selected (dense context), then the
+    whole PISA forward and its fused kernel at each keep ratio.  Prints one
+    JSON line holding every row."""
+    import dataclasses
+    import torch
+    from workloads import Config
+    import sparse_attention_diffusion_block_b200 as pisa
+    from torch.nn.functional import scaled_dot_product_attention as sdpa
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    rows = []
+
+    def timed(fn, reps=5):
+        fn()
+        torch.cuda.synchronize()
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            fn()
+        z.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(z) / reps
+
+    for L, grid in SWEEP_GRIDS.items():
+        cfg = Config(f"sweep{L}", "bf16", 1, 24, L, 128, 128, seed=5, keep_ratio=0.1, kind="grid",
+                     grid=grid, R=16, A=1.5)
+        q, k, v = generate(cfg, redraws={})
+        qd, kd, vd = (torch.from_numpy(x).to(dev).to(torch.bfloat16) for x in (q, k, v))
+        b, h, nb, d, B = cfg.batch, cfg.heads, cfg.nb, cfg.d, cfg.block
+        dense_flops = 4.0 * L * L * d * b * h
+        stats = pisa.block_stats(qd, kd, vd, B)
+        M = pisa.cov_norm(kd, vd, B, stats[1], stats[2], stats[3])
+        ws_f = torch.empty(max(pisa.fused_workspace_size(b, h, L, d, B), 16), dtype=torch.uint8, device=dev)
+        o = torch.empty_like(qd)
+        sdpa_ms = timed(lambda: sdpa(qd, kd, vd))
+        sel_all = torch.arange(nb, dtype=torch.int32, device=dev).expand(b, h, nb, nb).contiguous()
+        every_ms = timed(lambda: pisa.attn_fwd_with_sel(qd, kd, vd, B, stats[1], stats[2], stats[3], sel_all,
+                                                        out=o, workspace=ws_f))
+        rows.append({"L": L, "keep": 1.0, "torch_sdpa_ms": sdpa_ms, "pisa_every_block_ms": every_ms,
+                     "dense_TFLOP/s_sdpa": dense_flops / sdpa_ms / 1e9,
+                     "dense_TFLOP/s_pisa_every_block": dense_flops / every_ms / 1e9})
+        del sel_all
+        for keep in SWEEP_KEEP:
+            kk = pisa.keep_count(L, B, keep)
+            ws = torch.empty(pisa.workspace_size(b, h, L, d, B, kk), dtype=torch.uint8, device=dev)
+            fwd_ms = timed(lambda: pisa.attn_fwd(qd, kd, vd, B, keep, out=o, workspace=ws))
+            sel = pisa.select(stats[0], stats[1], M, L, B, kk)
+            fused_ms = timed(lambda: pisa.attn_fwd_with_sel(qd, kd, vd, B, stats[1], stats[2], stats[3], sel,
+                                                            out=o, workspace=ws_f))
+            torch.cuda.synchronize()
+            ex, ap_ = effective_flops(dataclasses.replace(cfg, keep_ratio=keep), sel.cpu().numpy())
+            rows.append({"L": L, "keep": keep, "k": kk, "forward_ms": fwd_ms, "fused_ms": fused_ms,
+                         "effective_TFLOP/s": (ex + ap_) / fwd_ms / 1e9,
+                         "speedup_vs_sdpa": sdpa_ms / fwd_ms})
+            del ws, sel
+        if pisa.device_status() != 0:
+            raise RuntimeError("device status set during the sweep")
+        del qd, kd, vd, stats, M, ws_f, o
+        torch.cuda.empty_cache()
+    print(json.dumps({"sweep": "PISA forward vs dense attention, 24 heads, d=128, block 128, bf16",
+                      "rows": rows}), flush=True)
+    return 0
+
+
 def _source_sha(paths):
     import hashlib
     h = hashlib.sha256()
@@ -270,6 +384,10 @@ def main():
                     help="seconds of oracle time for the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="sequence-length x density sweep (4K-32K tokens) instead of the bench line")
+    ap.add_argument("--no-dense-reference", action="store_true",
+                    help="skip the dense-attention context (every block selected; torch SDPA)")
     ap.add_argument("--e2e-chunk", type=int, default=2,
                     help="(batch, head) slices per chunk of the host-buffer pipeline")
     ap.add_argument("--heads", type=int, default=None,
@@ -282,6 +400,8 @@ def main():
         import dataclasses
         cfg = dataclasses.replace(cfg, heads=min(args.heads, cfg.heads))
 
+    if args.sweep:
+        return run_sweep(args)
     if args.impl == "reference":
         import oracle  # reference arm: the oracle as it stands
         return run_reference(args, cfg, oracle.keep_count(cfg.L, cfg.block, cfg.keep_ratio))
@@ -427,6 +547,10 @@ def main():
         stages[n] = ent
     stages["fused"]["TFLOP/s"] = achieved
 
+    dense = None
+    if rank == 0 and world == 1 and not args.no_dense_reference:
+        dense = dense_reference(pisa, cfg, qd, kd, vd, stats, fused_ms, ms)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tf, desc, threads, spent = cpu_oracle_sample(cfg, q, k, v, kk, args.cpu_budget)
@@ -446,6 +570,7 @@ def main():
             "roofline": roofline,
             "stages": stages,
             "cpu_baseline": cpu,
+            "dense_reference": dense,
             "e2e": e2e,
             "gpu_launches": K * pisa.launches("attn_fwd", tdt),
             "clocks": clocks.summary(),
