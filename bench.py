@@ -345,6 +345,23 @@ def run_sweep(args):
     return 0
 
 
+def max_over_ranks(x: float, dist, device) -> float:
+    """The maximum of ``x`` over all ranks (the slowest rank's time); ``x``
+    itself when not distributed."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_throughput(flops_per_rank: float, world: int, ms: float) -> float:
+    """Weak scaling: every rank runs the same workload, so the job moves
+    ``world`` times the per-rank FLOPs in the slowest rank's time."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 def _source_sha(paths):
     import hashlib
     h = hashlib.sha256()
@@ -487,12 +504,9 @@ def main():
     total_ms = t0.elapsed_time(t1)
     names = ["stats", "cov_norm", "select", "fused"]
     stage_ms = {n: sum(e[i].elapsed_time(e[i + 1]) for e in evs) / K for i, n in enumerate(names)}
-    if dist:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, dev)
     ms = total_ms / K
-    value = world * flops / (ms * 1e-3) / 1e12
+    value = whole_job_throughput(flops, world, ms)
 
     # end to end through the public API with host buffers: pisa_attn_fwd_host
     # copies chunks of heads in, computes and copies out, overlapping the three
@@ -516,14 +530,9 @@ def main():
             e2e_step()
         z.record()
         torch.cuda.synchronize()
-        e_ms = a.elapsed_time(z)
-        if dist:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e_ms /= K
+        e_ms = max_over_ranks(a.elapsed_time(z), dist, dev) / K
         in_bytes = sum(x.numel() * x.element_size() for x in (qd, kd, vd))
-        e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e_ms,
+        e2e = {"value": whole_job_throughput(flops, world, e_ms), "unit": "TFLOP/s", "ms_per_step": e_ms,
                "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out.numel() * out.element_size(),
                "api": f"pisa_attn_fwd_host, pinned host buffers, chunks of {args.e2e_chunk} heads"}
         del ws_host
