@@ -201,7 +201,7 @@ pisa_status pisa_attn_fwd_host(const void* q_host, const void* k_host, const voi
  *
  * Same arguments and results as pisa_attn_fwd_with_sel minus the workspace.
  * The scratch that pisa_attn_fwd_with_sel takes from the caller's workspace
- * (the tensor-core kernel's bf16 hi/lo copies of kbar, vsum and Hbar) lives
+ * (the tensor-core kernel's bf16 copies of kbar, vsum and Hbar) lives
  * instead in one device array of PISA_NOALLOC_SCRATCH_BYTES compiled into the
  * library; every GPU that loads the library holds that memory until the
  * process exits.

@@ -63,12 +63,13 @@ size_t stats_ws(const Shape& s) {
   return align_up((size_t)s.BH() * stats_chunks(s) * s.d * s.d * sizeof(float));
 }
 
-// bf16 hi/lo operands of the tensor-core fused kernel: centroid keys and
-// value sums [BH][2*nbp][d], Hbar transposed [BH][2*d][d].
+// bf16 operands of the tensor-core fused kernel: centroid keys [BH][nbp][d],
+// value sums [BH][nbp][d], Hbar transposed as hi/lo [BH][2*d][d].
 int padded_blocks(const Shape& s) { return (s.nb() + 127) / 128 * 128; }
 size_t fused_ws(const Shape& s) {
-  const size_t cent = align_up((size_t)s.BH() * 2 * padded_blocks(s) * s.d * 2);
-  return 2 * cent + align_up((size_t)s.BH() * 2 * s.d * s.d * 2);
+  const size_t keys = align_up((size_t)s.BH() * padded_blocks(s) * s.d * 2);
+  const size_t vals = align_up((size_t)s.BH() * padded_blocks(s) * s.d * 2);
+  return keys + vals + align_up((size_t)s.BH() * 2 * s.d * s.d * 2);
 }
 
 struct Carve {
@@ -255,16 +256,17 @@ pisa_status run_fused_sm100(const __nv_bfloat16* q, const __nv_bfloat16* k, cons
                             const float* hbar, const int32_t* sel, int kk, void* ws, cudaStream_t st) {
   const int nb = s.nb(), nbp = padded_blocks(s), BH = s.BH();
   char* w = static_cast<char*>(ws);
-  const size_t cent = align_up((size_t)BH * 2 * nbp * D * 2);
+  const size_t keys = align_up((size_t)BH * nbp * D * 2);
+  const size_t vals = align_up((size_t)BH * nbp * D * 2);
   __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(w);
-  __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(w + cent);
-  __nv_bfloat16* ht = reinterpret_cast<__nv_bfloat16*>(w + 2 * cent);
+  __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(w + keys);
+  __nv_bfloat16* ht = reinterpret_cast<__nv_bfloat16*>(w + keys + vals);
   const int elems = nbp * D > D * D ? nbp * D : D * D;
   prep_fused_operands_kernel<D><<<dim3((elems + 255) / 256, BH), 256, 0, st>>>(kbar, vsum, hbar, nb, nbp, kc, vc, ht);
   if (last_launch() != PISA_OK) return PISA_ERR_CUDA;
   CUtensorMap mQ, mK, mV, mKc, mVc, mH;
   if (!make_map(&mQ, q, D, s.L, BH, 128) || !make_map(&mK, k, D, s.L, BH, KB) || !make_map(&mV, v, D, s.L, BH, KB) ||
-      !make_map(&mKc, kc, D, 2 * nbp, BH, 128) || !make_map(&mVc, vc, D, 2 * nbp, BH, 128) ||
+      !make_map(&mKc, kc, D, nbp, BH, 128) || !make_map(&mVc, vc, D, nbp, BH, 128) ||
       !make_map(&mH, ht, D, 2 * D, BH, D))
     return PISA_ERR_CUDA;
   constexpr int G = 128 / KB;
