@@ -253,6 +253,15 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         L_[5] = tA;
         L_[6] = nA;
         L_[7] = nB;
+        // padding centroids [nb, nbp) count as selected in every mask, so the
+        // softmax masks a centroid column with one bit test
+        for (int w = nb >> 5; w < words; ++w) {
+          const uint32_t pad = (w << 5) >= nb ? 0xffffffffu : ~((1u << (nb & 31)) - 1u);
+          for (int g = 0; g < G; ++g) {
+            mA[g * words + w] |= pad;
+            mB[g * words + w] |= pad;
+          }
+        }
         mbar_arrive(&list_full[slot]);
 
         const PairPlan pl{(nA + G - 1) / G, (nB + G - 1) / G, nC / G, existsB, n_cent};
@@ -494,21 +503,35 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
               }
             }
           } else {
+            // centroid columns: masked when selected by this row's query block
+            // (or padding); the mask words are the same for every row group
+            // member, so the bit tests are uniform
             const int c0 = (u - pl.U()) * 128;
             const uint32_t* mw = msk + c0 / 32;
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-              const uint32_t bits = mw[w];
-#pragma unroll
-              for (int b = 0; b < 32; ++b) {
-                const int c = w * 32 + b;
-                const bool use = (c0 + c < nb) && !((bits >> b) & 1u);
-                const float v = use ? __uint_as_float(s[c]) : -INFINITY;
-                s[c] = __float_as_uint(v);
-                tmax = fmaxf(tmax, v);
-                if (c0 + c == nb - 1) x_tail = v;
-              }
+            const uint32_t bw[4] = {mw[0], mw[1], mw[2], mw[3]};
+            // a partial tail block's centroid stands for n_tail tokens, not
+            // block: read its logit before P overwrites S, to correct its mass
+            const int ct = nb - 1 - c0;
+            if (n_tail != a.block && ct >= 0 && ct < 128 && !((bw[ct >> 5] >> (ct & 31)) & 1u)) {
+              x_tail = __uint_as_float(tmem_ld1(sbase + ct));
+              tmem_wait_ld();
             }
+            float t0 = -INFINITY, t1 = -INFINITY, t2 = -INFINITY, t3 = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 128; c += 8) {
+              float v[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int cc = c + e;
+                v[e] = ((bw[cc >> 5] >> (cc & 31)) & 1u) ? -INFINITY : __uint_as_float(s[cc]);
+                s[cc] = __float_as_uint(v[e]);
+              }
+              t0 = fmax3(t0, v[0], v[1]);
+              t1 = fmax3(t1, v[2], v[3]);
+              t2 = fmax3(t2, v[4], v[5]);
+              t3 = fmax3(t3, v[6], v[7]);
+            }
+            tmax = fmax3(fmaxf(t0, t1), t2, t3);
           }
           // running max in log2 units; lazy rescale when it grows by more than 8
           const float m_new = fmaxf(m, tmax * c2);

@@ -31,12 +31,6 @@ struct StatsLayout {
   static constexpr size_t bytes() { return 1024 + kRing + kOnes + kSig + kRed + kBars + 16; }
 };
 
-__device__ __forceinline__ uint32_t tmem_ld1(uint32_t taddr) {
-  uint32_t r;
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
-  return r;
-}
-
 // Descriptor of an MN-major operand held as [rows][128] bf16 in two 64-column
 // swizzled blocks, rows = contraction dimension; k-step kk covers rows 16kk..16kk+15.
 __device__ __forceinline__ uint64_t desc_mn(uint32_t base, int rows, int kk) {
