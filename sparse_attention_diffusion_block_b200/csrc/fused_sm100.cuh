@@ -19,9 +19,12 @@
 //              o = (O + s beta q Hbar) / l.
 //   warp 8     producer: builds each pair's work list in shared memory, then
 //              streams Q tiles and a ring of 128-row operand tiles with TMA.
-//   warp 9     MMA issuer (one thread): S = Q K^T and O += P V (P from TMEM),
-//              ping-ponging the two tiles so that one tile's softmax overlaps
-//              the other tile's MMAs.
+//   warp 9     MMA issuer: S = Q K^T and O += P V (P from TMEM), ping-ponging
+//              the two tiles so that one tile's softmax overlaps the other
+//              tile's MMAs.  The whole warp runs the issue loop and one
+//              elected lane issues each instruction, which keeps the operands
+//              in warp-uniform registers (a lone lane in a divergent branch
+//              issues markedly slower).
 // Work list of a pair: the exact KV blocks of each tile (for 64-token blocks a
 // 128-row tile spans two query blocks: the union, with per-row-group bits),
 // blocks selected by both tiles first and in the same order, so those K/V
@@ -328,7 +331,10 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     }
    } else if (warp == 9) {
     // ================================================================ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the issue loop, so descriptors, slot indices and
+    // barrier waits are warp-uniform; one elected lane issues each tcgen05
+    // instruction.
+    {
       constexpr uint32_t idC = idesc_bf16(128, 128, false, false);  // every step is 128 keys
       constexpr uint32_t idH = idesc_bf16(128, D, false, false);
       constexpr uint32_t idO = idesc_bf16(128, D, false, true);
@@ -371,9 +377,9 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         auto issue_s = [&](int x, int u) -> bool {
           const uint32_t sc = tmem + x * 128;
           if (!((x == 1) && pl.shared(u)) && !take(ks)) return false;  // tile B reuses tile A's items when shared
-          for (int kk = 0; kk < D / 16; ++kk) mma_ss(sc, qdesc(x, kk), kdesc(ks, 128, kk), idC, kk > 0 ? 1u : 0u);
-          if (!((x == 0) && pl.shared(u))) mma_commit(&empty[ks]);
-          mma_commit(&s_full[x]);
+          for (int kk = 0; kk < D / 16; ++kk) mma_ss_warp(sc, qdesc(x, kk), kdesc(ks, 128, kk), idC, kk > 0 ? 1u : 0u);
+          if (!((x == 0) && pl.shared(u))) mma_commit_warp(&empty[ks]);
+          mma_commit_warp(&s_full[x]);
           return true;
         };
         auto issue_pv = [&](int x, int u) -> bool {
@@ -385,9 +391,9 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           // one V item per step: a 128-token value tile or 128 centroid value sums
           if (!((x == 1) && pl.shared(u)) && !take(vs)) return false;
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(oc, pa + kk * 8, vdesc(vs, 128, kk), idO, (!first_pv[x] || kk > 0) ? 1u : 0u);
+            mma_ts_warp(oc, pa + kk * 8, vdesc(vs, 128, kk), idO, (!first_pv[x] || kk > 0) ? 1u : 0u);
           first_pv[x] = false;
-          if (!((x == 0) && pl.shared(u))) mma_commit(&empty[vs]);
+          if (!((x == 0) && pl.shared(u))) mma_commit_warp(&empty[vs]);
           return true;
         };
         // before reusing S_x / O_x the previous epilogue of tile x must have read them
@@ -411,17 +417,17 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (!(ok = take(h0) && take(h1))) break;
         for (int x = 0; x < 1 + pl.existsB; ++x) {
           const uint32_t sc = tmem + x * 128;
-          for (int kk = 0; kk < D / 16; ++kk) mma_ss(sc, qdesc(x, kk), kdesc(h0, D, kk), idH, kk > 0 ? 1u : 0u);
-          for (int kk = 0; kk < D / 16; ++kk) mma_ss(sc, qdesc(x, kk), kdesc(h1, D, kk), idH, 1u);
-          mma_commit(&o_final[x]);
-          mma_commit(&q_empty[x]);
+          for (int kk = 0; kk < D / 16; ++kk) mma_ss_warp(sc, qdesc(x, kk), kdesc(h0, D, kk), idH, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) mma_ss_warp(sc, qdesc(x, kk), kdesc(h1, D, kk), idH, 1u);
+          mma_commit_warp(&o_final[x]);
+          mma_commit_warp(&q_empty[x]);
           ++epis[x];
         }
-        mma_commit(&empty[h0]);
-        mma_commit(&empty[h1]);
-        mbar_arrive(&list_empty[slot]);
+        mma_commit_warp(&empty[h0]);
+        mma_commit_warp(&empty[h1]);
+        if (lane == 0) mbar_arrive(&list_empty[slot]);
       }
-      mma_commit(mma_idle);
+      mma_commit_warp(mma_idle);
       volatile int never = 0;
       mbar_wait(mma_idle, 0, &never);
     }
@@ -453,6 +459,7 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const int qtile = L_[5] + x;
       const int* ent = L_ + 8 + x * G * a.kk;
       const int n_ent = L_[6 + x];
+      int ent_win = -1, ent_reg = 0;
       const uint32_t* msk = reinterpret_cast<const uint32_t*>(L_ + 8 + 2 * G * a.kk) + x * G * words + g * words;
       if (x == 0 || pl.existsB) {
         const int qrow = qtile * QT + row;
@@ -478,12 +485,19 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             // column half h (of KB columns) holds list entry G u + h; the keys of
             // that block this row may use: all of its tokens if the row's query
             // block selected it, none otherwise (or when the entry is absent)
+            // the tile's list entries sit in a 32-entry register window, one
+            // per lane, refilled from shared memory every 32 entries
+            if (((G * u) >> 5) != ent_win) {
+              ent_win = (G * u) >> 5;
+              const int idx = ent_win * 32 + lane;
+              ent_reg = idx < n_ent ? ent[idx] : 0;
+            }
             int nvalid[G];
 #pragma unroll
             for (int h = 0; h < G; ++h) {
               nvalid[h] = 0;
+              const int e = __shfl_sync(0xffffffffu, ent_reg, (G * u + h) & 31);
               if (G * u + h < n_ent) {
-                const int e = ent[G * u + h];
                 const int j = e & 0xFFFFFF;
                 if ((e >> (24 + g)) & 1) nvalid[h] = min(KB, a.L - j * KB);
               }
@@ -492,8 +506,15 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 #pragma unroll
             for (int h = 0; h < G; ++h) whole = whole && nvalid[h] == KB;
             if (__all_sync(0xffffffffu, whole)) {
+              float t0 = -INFINITY, t1 = -INFINITY, t2 = -INFINITY, t3 = -INFINITY;
 #pragma unroll
-              for (int c = 0; c < 128; ++c) tmax = fmaxf(tmax, __uint_as_float(s[c]));
+              for (int c = 0; c < 128; c += 8) {
+                t0 = fmax3(t0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+                t1 = fmax3(t1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+                t2 = fmax3(t2, __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));
+                t3 = fmax3(t3, __uint_as_float(s[c + 6]), __uint_as_float(s[c + 7]));
+              }
+              tmax = fmax3(fmaxf(t0, t1), t2, t3);
             } else {
 #pragma unroll
               for (int c = 0; c < 128; ++c) {
