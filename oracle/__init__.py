@@ -26,6 +26,11 @@ s qbar_i.kbar_j + ln(n_j + s ||qbar_i|| M_j); R8 queries pooled by block mean;
 R9 k = clamp(ceil(rho nb - 1e-9), 1, nb); R10 ties to the smaller index, no
 forced block; R11 non-causal; R12 true counts n_j for a partial tail block.
 
+Variants of three readings, kept beside the defaults for comparison: the
+spectral norm for M_j (R6), the pooled score without the covariance term
+(R7), and the un-hybridised first-order term with each unselected block's own
+H_j (the summary's starting point before Hbar).
+
 Parity unpinned: the routing score formula (R7) and the norm choice (R6).
 Nothing on the pages fixes them; the tests pin their structure (V = 0 reduces
 the score to pooled block-sparse routing; permutation invariance) but not the
@@ -39,7 +44,9 @@ from .pisa_ref import (  # noqa: F401
     first_order_blocks,
     hbar_mean,
     cov_norm,
+    cov_norm_spectral,
     route_scores,
+    route_scores_pooled,
     select_topk,
     pisa_rows,
     pisa_head,

@@ -105,6 +105,24 @@ def cov_norm(H: np.ndarray, Hbar: np.ndarray) -> np.ndarray:
     return np.sqrt((diff * diff).sum(axis=(1, 2)))
 
 
+def cov_norm_spectral(H: np.ndarray, Hbar: np.ndarray) -> np.ndarray:
+    """M_j = ||H_j - Hbar||_2 read as the spectral norm (largest singular
+    value): the other reading of the matrix 2-norm in the covariance-aware
+    routing paragraph (gist.science summary, section 2).  A variant of reading
+    R6, not the default."""
+    diff = H - Hbar[None, :, :]
+    return np.linalg.norm(diff, ord=2, axis=(1, 2))
+
+
+def route_scores_pooled(qbar: np.ndarray, kbar: np.ndarray, n: np.ndarray, s: float) -> np.ndarray:
+    """Routing score without the covariance term: s qbar_i . kbar_j + ln n_j,
+    the log of the block's zeroth-order softmax mass (the attention part of
+    Score_{t,j} alone; a variant of reading R7, plain pooled block-sparse
+    routing)."""
+    att = s * (qbar @ kbar.T)
+    return att + np.log(n)[None, :]
+
+
 def route_scores(qbar: np.ndarray, kbar: np.ndarray, M: np.ndarray, n: np.ndarray, s: float) -> np.ndarray:
     """Routing score of KV block j for query block i (reading R7; parity unpinned).
 
@@ -133,9 +151,16 @@ def select_topk(scores: np.ndarray, kk: int) -> np.ndarray:
     return sel
 
 
-def pisa_rows(q, k, v, B, sel, kbar, vsum, n, Hbar, rows, s, return_parts=False):
+def pisa_rows(q, k, v, B, sel, kbar, vsum, n, Hbar, rows, s, return_parts=False, H_blocks=None):
     """Output rows o_t = N_t / D_t for the query tokens ``rows`` (gist.science
     summary, section 2, core algorithm).
+
+    With ``H_blocks`` (the [nb, d, d] block-wise matrices H_j) the first-order
+    term is the un-hybridised one the summary's hybrid-order paragraph starts
+    from: every unselected block keeps its own H_j,
+      N_t = ... + s sum_{j in U} e^{y_{t,j}} (q_t H_j)
+    instead of s beta_t (q_t Hbar) (a variant for the accuracy / cost
+    comparison; it costs |U| d^2 per query row).
 
     For t in query block i (S = S_i, U = U_i the complement):
       x_{t,n} = s q_t . k_n      for every token n of every block in S
@@ -170,7 +195,14 @@ def pisa_rows(q, k, v, B, sel, kbar, vsum, n, Hbar, rows, s, return_parts=False)
         exact_den = ex.sum(axis=1)
         D = exact_den + ey @ n[U]
         beta = ey.sum(axis=1)
-        N = ex @ v[cols] + ey @ vsum[U] + s * beta[:, None] * (qi @ Hbar)
+        if H_blocks is None:
+            first = s * beta[:, None] * (qi @ Hbar)
+        else:
+            first = np.zeros((len(pick), v.shape[1]))
+            for c, j in enumerate(U):
+                first += ey[:, c:c + 1] * (qi @ H_blocks[j])
+            first *= s
+        N = ex @ v[cols] + ey @ vsum[U] + first
         if not np.all(D > 0):
             raise AssertionError("D_t must be positive")
         out[pick] = N / D[:, None]
@@ -181,12 +213,18 @@ def pisa_rows(q, k, v, B, sel, kbar, vsum, n, Hbar, rows, s, return_parts=False)
     return out
 
 
-def pisa_head(q, k, v, B, kk, s=None, rows=None):
+def pisa_head(q, k, v, B, kk, s=None, rows=None, norm="frobenius", route="covariance",
+              first_order="hybrid"):
     """The whole method on one (batch, head): stats, Hbar, M, scores, S, output.
 
     q, k, v: [L, d] arrays (promoted to float64).  ``rows`` limits the output
     to the given query tokens (all rows when None).  Returns a dict of every
     intermediate so that each stage can be compared on its own.
+
+    Variants (defaults are readings R6, R7 and the pages' hybrid term):
+    ``norm`` "frobenius" or "spectral" for M_j; ``route`` "covariance" or
+    "pooled" (no M term); ``first_order`` "hybrid" (Hbar) or "blockwise"
+    (each unselected block's own H_j).
     """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
@@ -197,12 +235,25 @@ def pisa_head(q, k, v, B, kk, s=None, rows=None):
     qbar, kbar, vsum, n = block_stats(q, k, v, B)
     H = first_order_blocks(k, v, B, kbar)
     Hbar = hbar_mean(H)
-    M = cov_norm(H, Hbar)
-    scores = route_scores(qbar, kbar, M, n, s)
+    if norm == "frobenius":
+        M = cov_norm(H, Hbar)
+    elif norm == "spectral":
+        M = cov_norm_spectral(H, Hbar)
+    else:
+        raise ValueError(norm)
+    if route == "covariance":
+        scores = route_scores(qbar, kbar, M, n, s)
+    elif route == "pooled":
+        scores = route_scores_pooled(qbar, kbar, n, s)
+    else:
+        raise ValueError(route)
     sel = select_topk(scores, kk)
     if rows is None:
         rows = np.arange(L)
-    out = pisa_rows(q, k, v, B, sel, kbar, vsum, n, Hbar, rows, s)
+    if first_order not in ("hybrid", "blockwise"):
+        raise ValueError(first_order)
+    out = pisa_rows(q, k, v, B, sel, kbar, vsum, n, Hbar, rows, s,
+                    H_blocks=H if first_order == "blockwise" else None)
     return dict(out=out, sel=sel, qbar=qbar, kbar=kbar, vsum=vsum, n=n,
                 H=H, Hbar=Hbar, M=M, scores=scores, s=s)
 

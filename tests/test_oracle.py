@@ -307,3 +307,123 @@ def test_keep_count_on_the_workloads():
 def test_block_bounds_partial_tail():
     s, e = oracle.block_bounds(300, 128)
     assert s.tolist() == [0, 128, 256] and e.tolist() == [128, 256, 300]
+
+
+# ---------------------------------------------------------------- variants of the readings
+
+
+def _rank_one_case(L=200, B=20, d=8, seed=9):
+    """Keys k_n = c_j + a_n e with one unit direction e and per-block centred
+    scalars a_n: every H_j - Hbar is then e (w_j - wbar)^T, of rank one, with
+    w_j = sum_n a_n v_n."""
+    rng = np.random.default_rng(seed)
+    nb = L // B
+    e = rng.standard_normal(d)
+    e /= np.linalg.norm(e)
+    a = rng.standard_normal(L)
+    for j in range(nb):
+        a[j * B:(j + 1) * B] -= a[j * B:(j + 1) * B].mean()
+    k = rng.standard_normal((nb, d))[np.arange(L) // B] + a[:, None] * e[None, :]
+    v = rng.standard_normal((L, d))
+    w = np.stack([(a[j * B:(j + 1) * B, None] * v[j * B:(j + 1) * B]).sum(axis=0) for j in range(nb)])
+    return k, v, w
+
+
+def test_spectral_norm_of_rank_one_deviations_is_their_vector_norm():
+    """Rank-one H_j - Hbar: spectral norm = Frobenius norm = ||w_j - wbar||."""
+    k, v, w = _rank_one_case()
+    B = 20
+    kbar = oracle.block_stats(k, k, v, B)[1]
+    H = oracle.first_order_blocks(k, v, B, kbar)
+    Hbar = oracle.hbar_mean(H)
+    want = np.linalg.norm(w - w.mean(axis=0), axis=1)
+    np.testing.assert_allclose(oracle.cov_norm_spectral(H, Hbar), want, rtol=1e-10)
+    np.testing.assert_allclose(oracle.cov_norm(H, Hbar), want, rtol=1e-10)
+
+
+def test_spectral_norm_bounds_for_generic_blocks():
+    """||A||_2 <= ||A||_F <= sqrt(rank) ||A||_2, and ||A||_2 >= the largest
+    column norm of A (A e_c for a unit vector e_c)."""
+    rng = np.random.default_rng(21)
+    q, k, v = rng.standard_normal((3, 240, 12))
+    B = 24
+    kbar = oracle.block_stats(q, k, v, B)[1]
+    H = oracle.first_order_blocks(k, v, B, kbar)
+    Hbar = oracle.hbar_mean(H)
+    spec, frob = oracle.cov_norm_spectral(H, Hbar), oracle.cov_norm(H, Hbar)
+    assert (spec <= frob * (1 + 1e-12)).all()
+    assert (frob <= math.sqrt(12) * spec * (1 + 1e-12)).all()
+    col = np.sqrt(((H - Hbar) ** 2).sum(axis=1)).max(axis=1)
+    assert (spec >= col * (1 - 1e-12)).all()
+    assert (spec < frob).any()  # not the Frobenius norm again
+
+
+@pytest.mark.parametrize("L,B,kk", [(500, 50, 3), (256, 32, 1)])
+def test_pooled_routing_is_brute_force_top_k(L, B, kk):
+    """Pooled score s qbar.kbar + ln n_j, selection checked against a pure
+    Python sort; with V = 0 (M = 0) the covariance score equals it."""
+    rng = np.random.default_rng(L + kk)
+    q, k = rng.standard_normal((2, L, 16))
+    s = 0.25
+    qbar, kbar, _, n = oracle.block_stats(q, k, k, B)
+    sc = oracle.route_scores_pooled(qbar, kbar, n, s)
+    sel = oracle.select_topk(sc, kk)
+    for i in range(len(qbar)):
+        pairs = [(-(s * sum(qbar[i][a] * kbar[j][a] for a in range(16)) + math.log(n[j])), j)
+                 for j in range(len(kbar))]
+        assert sorted(j for _, j in sorted(pairs)[:kk]) == list(sel[i])
+    zeros = np.zeros((len(kbar),))
+    np.testing.assert_allclose(oracle.route_scores(qbar, kbar, zeros, n, s), sc, rtol=0, atol=1e-12)
+
+
+def _blockwise_slope(shared):
+    B = 12
+    sel = np.array([[i, (i + 3) % 8] for i in range(8)])
+    sel.sort(axis=1)
+    eps = np.array([1e-1, 3e-2, 1e-2, 3e-3, 1e-3])
+    errs = []
+    for e in eps:
+        q, k, v = _taylor_case(e, shared)
+        s = 1 / math.sqrt(q.shape[1])
+        qbar, kbar, vsum, n = oracle.block_stats(q, k, v, B)
+        H = oracle.first_order_blocks(k, v, B, kbar)
+        o = oracle.pisa_rows(q, k, v, B, sel, kbar, vsum, n, oracle.hbar_mean(H), np.arange(q.shape[0]), s,
+                             H_blocks=H)
+        errs.append(np.abs(o - oracle.dense_attention(q, k, v)).max())
+    return np.polyfit(np.log(eps), np.log(errs), 1)[0]
+
+
+def test_blockwise_first_order_is_second_order_for_generic_blocks():
+    """Each unselected block keeps its own H_j: a true first-order Taylor
+    expansion per block, so the error is O(eps^2) even when the H_j differ
+    (where the hybrid Hbar term is only O(eps))."""
+    assert _blockwise_slope(shared=False) == pytest.approx(2.0, abs=0.15)
+
+
+def test_blockwise_equals_hybrid_when_every_block_shares_hbar():
+    q, k, v = _taylor_case(1e-2, shared=True)
+    B = 12
+    s = 1 / math.sqrt(q.shape[1])
+    sel = np.sort(np.array([[i, (i + 5) % 8] for i in range(8)]), axis=1)
+    qbar, kbar, vsum, n = oracle.block_stats(q, k, v, B)
+    H = oracle.first_order_blocks(k, v, B, kbar)
+    Hbar = oracle.hbar_mean(H)
+    rows = np.arange(q.shape[0])
+    a = oracle.pisa_rows(q, k, v, B, sel, kbar, vsum, n, Hbar, rows, s)
+    b = oracle.pisa_rows(q, k, v, B, sel, kbar, vsum, n, Hbar, rows, s, H_blocks=H)
+    np.testing.assert_allclose(b, a, rtol=0, atol=1e-12)
+
+
+def test_head_variants_run_and_differ_only_where_expected():
+    rng = np.random.default_rng(5)
+    q, k, v = rng.standard_normal((3, 300, 16))
+    base = oracle.pisa_head(q, k, v, 30, 3)
+    spec = oracle.pisa_head(q, k, v, 30, 3, norm="spectral")
+    pooled = oracle.pisa_head(q, k, v, 30, 3, route="pooled")
+    block = oracle.pisa_head(q, k, v, 30, 3, first_order="blockwise")
+    np.testing.assert_array_equal(block["sel"], base["sel"])          # routing untouched
+    assert not np.allclose(block["out"], base["out"])                # first-order term changed
+    assert (spec["M"] <= base["M"] * (1 + 1e-12)).all()
+    np.testing.assert_allclose(pooled["M"], base["M"])                # M computed, not used
+    with pytest.raises(ValueError):
+        oracle.pisa_head(q, k, v, 30, 3, norm="nuclear")
