@@ -401,6 +401,9 @@ def main():
                     help="seconds of oracle time for the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--route", default="covariance", choices=["covariance", "pooled", "spectral"],
+                    help="routing variant: the default covariance score with the Frobenius norm, "
+                         "the pooled score, or the covariance score with the spectral norm")
     ap.add_argument("--sweep", action="store_true",
                     help="sequence-length x density sweep (4K-32K tokens) instead of the bench line")
     ap.add_argument("--no-dense-reference", action="store_true",
@@ -412,6 +415,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.route != "covariance":
+        args.no_e2e = True  # the host-buffer entry point runs the default routing
     cfg = workload_config(args.workload)
     if args.heads is not None:
         import dataclasses
@@ -462,20 +467,31 @@ def main():
         if ev: ev[0].record()
         pisa.block_stats(qd, kd, vd, B, workspace=ws_stats, out=stats)
         if ev: ev[1].record()
-        pisa.cov_norm(kd, vd, B, stats[1], stats[2], stats[3], out=M)
+        if args.route == "covariance":
+            pisa.cov_norm(kd, vd, B, stats[1], stats[2], stats[3], out=M)
+        elif args.route == "spectral":
+            # variant: M_j as the spectral norm, from the stored block matrices
+            Hb = pisa.block_first_order(kd, vd, B, stats[1], stats[2])
+            pisa.cov_norm_spectral(Hb, stats[3], L, B, out=M)
+            del Hb
         if ev: ev[2].record()
-        pisa.select(stats[0], stats[1], M, L, B, kk, out=sel)
+        if args.route == "pooled":
+            pisa.select_route(stats[0], stats[1], None, L, B, kk, route="pooled", out=sel)
+        else:
+            pisa.select(stats[0], stats[1], M, L, B, kk, out=sel)
         if ev: ev[3].record()
         pisa.attn_fwd_with_sel(qd, kd, vd, B, stats[1], stats[2], stats[3], sel, out=out, workspace=ws_fused)
         if ev: ev[4].record()
 
     # correctness guard: the staged calls equal the one-shot entry point
     forward()
-    ref_out = pisa.attn_fwd(qd, kd, vd, B, cfg.keep_ratio, workspace=ws_all)
+    if args.route == "covariance":
+        ref_out = pisa.attn_fwd(qd, kd, vd, B, cfg.keep_ratio, workspace=ws_all)
+        torch.cuda.synchronize()
+        if not torch.equal(ref_out, out):
+            raise RuntimeError("staged forward differs from pisa_attn_fwd")
+        del ref_out
     torch.cuda.synchronize()
-    if not torch.equal(ref_out, out):
-        raise RuntimeError("staged forward differs from pisa_attn_fwd")
-    del ref_out
     status = pisa.device_status()
     if status != 0:
         raise RuntimeError(f"device status {pisa.status_string(status)}")
@@ -575,6 +591,7 @@ def main():
             "config": {"workload": describe(cfg, kk), "global_batch": world * cfg.batch,
                        "seq_len": cfg.L, "parallelism": f"replicas x{world} (one full forward per GPU)",
                        "l2": f"inputs {3 * qd.numel() * qd.element_size() / 1e9:.2f} GB > L2 126 MB",
+                       "route": args.route,
                        "flops_exact": exact, "flops_approx": approx},
             "roofline": roofline,
             "stages": stages,

@@ -61,6 +61,12 @@ typedef enum pisa_dtype {
   PISA_FP32 = 1
 } pisa_dtype;
 
+/* Routing score used by pisa_select_route. */
+typedef enum pisa_route {
+  PISA_ROUTE_COVARIANCE = 0,  /* s qbar.kbar + ln(n_j + s ||qbar|| M_j): the default   */
+  PISA_ROUTE_POOLED = 1       /* s qbar.kbar + ln n_j: no covariance term (M unused) */
+} pisa_route;
+
 /* Text of a status code (static storage, never NULL). */
 const char* pisa_status_string(pisa_status status);
 
@@ -120,6 +126,27 @@ pisa_status pisa_block_first_order(const void* k, const void* v, pisa_dtype dtyp
 pisa_status pisa_select(const float* qbar, const float* kbar, const float* M,
                         int batch, int heads, int L, int d, int block, int k,
                         int32_t* sel, void* stream);
+
+/* Routing with a chosen score (variants of the routing reading, for
+ * comparison; gist.science summary, section 2, covariance-aware routing).
+ * PISA_ROUTE_COVARIANCE is exactly pisa_select.  PISA_ROUTE_POOLED drops the
+ * covariance term (M_j = 0): score = s qbar_i . kbar_j + ln n_j, plain pooled
+ * block-sparse routing; M is not read and may be NULL.  Any other route value
+ * returns PISA_ERR_INVALID_ARG. */
+pisa_status pisa_select_route(const float* qbar, const float* kbar, const float* M,
+                              int batch, int heads, int L, int d, int block, int k,
+                              pisa_route route, int32_t* sel, void* stream);
+
+/* Covariance norm read as the spectral norm (gist.science summary, section
+ * 2: ||H_j - Hbar||_2 as the largest singular value; the default,
+ * pisa_cov_norm, reads it as the Frobenius norm).  H: the block-wise
+ * matrices of pisa_block_first_order [batch, heads, nb, d, d] float32; hbar
+ * from pisa_block_stats; M [batch, heads, nb] float32.  One CTA per block forms
+ * G = (H_j - Hbar)^T (H_j - Hbar) and runs power iteration on it until its
+ * Rayleigh quotient changes by less than 1e-7 relative (at most 4000 steps);
+ * M_j = sqrt(lambda_max(G)), float32. */
+pisa_status pisa_cov_norm_spectral(const float* H, const float* hbar, int batch, int heads, int L,
+                                   int d, int block, float* M, void* stream);
 
 /* The fused forward for a given selection (gist.science summary, section 2:
  * core algorithm, N_t equation; hardware implementation phases 1-3).  For

@@ -6,7 +6,8 @@ memory and streams.  There is no CPU fallback: importing this module fails
 loudly when the library has not been built.
 
 Entry points mirror the C names (without the ``pisa_`` prefix):
-block_stats, cov_norm, block_first_order, select, attn_fwd_with_sel, attn_fwd,
+block_stats, cov_norm, cov_norm_spectral, block_first_order, select, select_route,
+attn_fwd_with_sel, attn_fwd,
 attn_fwd_host, attn_fwd_with_sel_noalloc, keep_count, workspace_size, stats_workspace_size,
 fused_workspace_size, host_workspace_size, device_status, status_string.
 """
@@ -38,6 +39,8 @@ PISA_ERR_TIMEOUT = -5
 PISA_ERR_DEVICE_CHECK = -6
 PISA_BF16 = 0
 PISA_FP32 = 1
+PISA_ROUTE_COVARIANCE = 0
+PISA_ROUTE_POOLED = 1
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # PISA_NOALLOC_SCRATCH_BYTES
 
 EXPORTS = (
@@ -45,7 +48,7 @@ EXPORTS = (
     "pisa_fused_workspace_size", "pisa_workspace_size", "pisa_block_stats", "pisa_cov_norm",
     "pisa_block_first_order", "pisa_select", "pisa_attn_fwd_with_sel", "pisa_attn_fwd",
     "pisa_device_status", "pisa_attn_fwd_with_sel_noalloc", "pisa_host_workspace_size",
-    "pisa_attn_fwd_host",
+    "pisa_attn_fwd_host", "pisa_select_route", "pisa_cov_norm_spectral",
 )
 
 _p = ctypes.c_void_p
@@ -78,6 +81,8 @@ _lib_fwd_sel_noalloc = _sig("pisa_attn_fwd_with_sel_noalloc", _i, _p, _p, _p, _p
 _lib_fwd = _sig("pisa_attn_fwd", _i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p, _z, _p)
 _lib_device_status = _sig("pisa_device_status", _i, _p, _i)
 _lib_host_ws = _sig("pisa_host_workspace_size", _z, _i, _i, _i, _i, _i, _i, _i, _i)
+_lib_select_route = _sig("pisa_select_route", _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _p)
+_lib_cov_spectral = _sig("pisa_cov_norm_spectral", _i, _p, _p, _i, _i, _i, _i, _i, _p, _p)
 _lib_fwd_host = _sig("pisa_attn_fwd_host", _i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _i, _p, _z, _p)
 
 
@@ -201,6 +206,29 @@ def select(qbar, kbar, M, L, block, k, stream=None, out=None):
     _check(_lib_select(_ptr(qbar), _ptr(kbar), _ptr(M), b, h, L, d, block, k, _ptr(sel),
                        _stream(stream)), "pisa_select")
     return sel
+
+
+def select_route(qbar, kbar, M, L, block, k, route="covariance", stream=None, out=None):
+    """Routing with a chosen score: "covariance" (pisa_select) or "pooled"
+    (no covariance term; ``M`` may be None)."""
+    code = {"covariance": PISA_ROUTE_COVARIANCE, "pooled": PISA_ROUTE_POOLED}[route]
+    _need_cuda(qbar, kbar, *(() if M is None else (M,)))
+    b, h, nb, d = qbar.shape
+    sel = out if out is not None else torch.empty(b, h, nb, k, dtype=torch.int32, device=qbar.device)
+    _check(_lib_select_route(_ptr(qbar), _ptr(kbar), _ptr(M), b, h, L, d, block, k, code, _ptr(sel),
+                             _stream(stream)), "pisa_select_route")
+    return sel
+
+
+def cov_norm_spectral(H, hbar, L, block, stream=None, out=None):
+    """M_j = ||H_j - Hbar||_2 (largest singular value) from the block-wise
+    matrices of block_first_order."""
+    _need_cuda(H, hbar)
+    b, h, nb, d, _ = H.shape
+    M = out if out is not None else torch.empty(b, h, nb, dtype=torch.float32, device=H.device)
+    _check(_lib_cov_spectral(_ptr(H), _ptr(hbar), b, h, L, d, block, _ptr(M), _stream(stream)),
+           "pisa_cov_norm_spectral")
+    return M
 
 
 def attn_fwd_with_sel(q, k, v, block, kbar, vsum, hbar, sel, out=None, workspace=None, stream=None):

@@ -10,6 +10,7 @@
 #include "common.cuh"
 #include "fused_simt.cuh"
 #include "fused_sm100.cuh"
+#include "route_variants.cuh"
 #include "select.cuh"
 #include "stats_simt.cuh"
 #include "stats_sm100.cuh"
@@ -593,6 +594,37 @@ pisa_status pisa_select(const float* qbar, const float* kbar, const float* M, in
   cudaStream_t st = (cudaStream_t)stream;
   return d == 128 ? run_select<128>(qbar, kbar, M, s, k, sel, st)
                   : run_select<64>(qbar, kbar, M, s, k, sel, st);
+}
+
+pisa_status pisa_select_route(const float* qbar, const float* kbar, const float* M, int batch, int heads, int L,
+                              int d, int block, int k, pisa_route route, int32_t* sel, void* stream) {
+  if (route == PISA_ROUTE_COVARIANCE) return pisa_select(qbar, kbar, M, batch, heads, L, d, block, k, sel, stream);
+  if (route != PISA_ROUTE_POOLED) return PISA_ERR_INVALID_ARG;
+  const Shape s{batch, heads, L, d, block};
+  if (pisa_status e = check_shape(s)) return e;
+  if (k < 1 || k > s.nb()) return PISA_ERR_INVALID_ARG;
+  if (!all_ok(qbar, kbar) || sel == nullptr || (reinterpret_cast<uintptr_t>(sel) & 3u)) return PISA_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  return d == 128 ? run_select<128>(qbar, kbar, nullptr, s, k, sel, st)
+                  : run_select<64>(qbar, kbar, nullptr, s, k, sel, st);
+}
+
+pisa_status pisa_cov_norm_spectral(const float* H, const float* hbar, int batch, int heads, int L, int d,
+                                   int block, float* M, void* stream) {
+  const Shape s{batch, heads, L, d, block};
+  if (pisa_status e = check_shape(s)) return e;
+  if (!all_ok(H, hbar, M)) return PISA_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (d == 128) {
+    const size_t smem = (2 * 128 * 128 + 2 * 128 + 16) * sizeof(float);
+    if (!set_smem(cov_spectral_kernel<128>, smem)) return PISA_ERR_CUDA;
+    cov_spectral_kernel<128><<<dim3(s.nb(), s.BH()), kSpectralThreads, smem, st>>>(H, hbar, s.nb(), M);
+  } else {
+    const size_t smem = (2 * 64 * 64 + 2 * 64 + 16) * sizeof(float);
+    if (!set_smem(cov_spectral_kernel<64>, smem)) return PISA_ERR_CUDA;
+    cov_spectral_kernel<64><<<dim3(s.nb(), s.BH()), kSpectralThreads, smem, st>>>(H, hbar, s.nb(), M);
+  }
+  return last_launch();
 }
 
 pisa_status pisa_attn_fwd_with_sel(const void* q, const void* k, const void* v, void* out, pisa_dtype dtype,

@@ -3,6 +3,8 @@
 // routing).  For query block i of a (batch, head):
 //   score_{i,j} = s qbar_i . kbar_j + ln(n_j + s ||qbar_i||_2 M_j)
 //   sel[i]      = the k largest scores, exact ties to the smaller j, ascending.
+// With M == nullptr the covariance term drops out (M_j = 0): score =
+// s qbar_i . kbar_j + ln n_j, plain pooled block-sparse routing.
 #pragma once
 
 #include "common.cuh"
@@ -66,7 +68,7 @@ select_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
     }
     if (threadIdx.x < KT) {
       const int j = j0 + threadIdx.x;
-      mj[threadIdx.x] = (j < nb) ? M[(size_t)bh * nb + j] : 0.f;
+      mj[threadIdx.x] = (j < nb && M != nullptr) ? M[(size_t)bh * nb + j] : 0.f;
       nj[threadIdx.x] = (j < nb) ? (float)min(B, L - j * B) : 1.f;
     }
     __syncthreads();

@@ -140,3 +140,22 @@ def test_host_entry_point_validates_before_any_cuda_call(lib):
     assert call(a12=None) == lib.PISA_ERR_WORKSPACE
     assert call(a13=ctypes.c_size_t(4096)) == lib.PISA_ERR_WORKSPACE
     assert call(a12=MISALIGNED) == lib.PISA_ERR_INVALID_ARG
+
+
+def test_routing_variant_entry_points_validate(lib):
+    raw = lib.raw_lib()
+    # unknown route value
+    assert raw.pisa_select_route(FAKE, FAKE, None, 1, 1, 1000, 128, 128, 2, 7, FAKE, None) == \
+        lib.PISA_ERR_INVALID_ARG
+    # the pooled route reads no M, covariance needs it
+    assert raw.pisa_select_route(None, FAKE, None, 1, 1, 1000, 128, 128, 2, lib.PISA_ROUTE_POOLED, FAKE,
+                                 None) == lib.PISA_ERR_INVALID_ARG
+    assert raw.pisa_select_route(FAKE, FAKE, None, 1, 1, 1000, 128, 128, 2, lib.PISA_ROUTE_COVARIANCE, FAKE,
+                                 None) == lib.PISA_ERR_INVALID_ARG
+    assert raw.pisa_select_route(FAKE, FAKE, None, 1, 1, 1000, 128, 128, 9, lib.PISA_ROUTE_POOLED, FAKE,
+                                 None) == lib.PISA_ERR_INVALID_ARG      # k > nb
+    # spectral norm: null H, unsupported d, misaligned M
+    assert raw.pisa_cov_norm_spectral(None, FAKE, 1, 1, 1000, 128, 128, FAKE, None) == lib.PISA_ERR_INVALID_ARG
+    assert raw.pisa_cov_norm_spectral(FAKE, FAKE, 1, 1, 1000, 96, 128, FAKE, None) == lib.PISA_ERR_UNSUPPORTED
+    assert raw.pisa_cov_norm_spectral(FAKE, FAKE, 1, 1, 1000, 128, 128, MISALIGNED, None) == \
+        lib.PISA_ERR_INVALID_ARG

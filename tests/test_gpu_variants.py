@@ -1,0 +1,116 @@
+"""GPU parity of the routing variants against the fp64 oracle: the pooled
+score without the covariance term (pisa_select_route) and the spectral-norm
+covariance norm (pisa_cov_norm_spectral).  Selections are compared on every
+row whose k-th and (k+1)-th oracle scores are at least 1e-3 apart (the
+generators' near-tie guard covers the default reading only); the output is
+compared for the GPU's own selection, row by row, against the oracle."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from workloads import small_config
+from parity_util import assert_output_close, assert_stat_close, inputs, to_device
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    small_config("variant_b128", L=1500, d=128, block=128, heads=2, keep_ratio=0.25, seed=51),
+    small_config("variant_b64_d64", L=1000, d=64, block=64, heads=2, keep_ratio=0.3, seed=52),
+    small_config("variant_ragged", L=1300, d=128, block=64, heads=1, keep_ratio=0.15, seed=53),
+]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    torch.cuda.init()
+
+
+def _compare_selection(gpu_sel, scores, kk, what, min_gap=1e-3):
+    ref = oracle.select_topk(scores, kk)
+    compared = 0
+    for i in range(scores.shape[0]):
+        top = np.sort(scores[i])[::-1]
+        if kk < len(top) and top[kk - 1] - top[kk] < min_gap:
+            continue
+        np.testing.assert_array_equal(gpu_sel[i], ref[i], err_msg=f"{what} row {i}")
+        compared += 1
+    assert compared >= 0.8 * scores.shape[0], f"{what}: only {compared} rows away from near-ties"
+
+
+def _check_output(lib, cfg, q, k, v, qd, kd, vd, stats, sel, b, h, what):
+    out = lib.attn_fwd_with_sel(qd, kd, vd, cfg.block, stats[1], stats[2], stats[3], sel)
+    torch.cuda.synchronize()
+    qq, kk_, vv = (x[b, h].astype(np.float64) for x in (q, k, v))
+    s = 1.0 / math.sqrt(cfg.d)
+    qbar, kbar, vsum, n = oracle.block_stats(qq, kk_, vv, cfg.block)
+    Hbar = oracle.hbar_mean(oracle.first_order_blocks(kk_, vv, cfg.block, kbar))
+    ref = oracle.pisa_rows(qq, kk_, vv, cfg.block, sel[b, h].cpu().numpy(), kbar, vsum, n, Hbar,
+                           np.arange(cfg.L), s)
+    assert_output_close(out[b, h].float().cpu().numpy(), ref, cfg.dtype, what)
+
+
+@pytest.mark.parametrize("cfg", CASES, ids=lambda c: c.name)
+def test_pooled_routing(lib, cfg):
+    q, k, v = inputs(cfg, redraws={})
+    qd, kd, vd = (to_device(x, cfg.dtype) for x in (q, k, v))
+    kk = lib.keep_count(cfg.L, cfg.block, cfg.keep_ratio)
+    stats = lib.block_stats(qd, kd, vd, cfg.block)
+    sel = lib.select_route(stats[0], stats[1], None, cfg.L, cfg.block, kk, route="pooled")
+    torch.cuda.synchronize()
+    assert lib.device_status() == 0
+    s = 1.0 / math.sqrt(cfg.d)
+    for b in range(cfg.batch):
+        for h in range(cfg.heads):
+            qbar, kbar, _, n = oracle.block_stats(*(x[b, h].astype(np.float64) for x in (q, k, v)), cfg.block)
+            scores = oracle.route_scores_pooled(qbar, kbar, n, s)
+            _compare_selection(sel[b, h].cpu().numpy(), scores, kk, f"{cfg.name}[{b},{h}] pooled")
+            _check_output(lib, cfg, q, k, v, qd, kd, vd, stats, sel, b, h, f"{cfg.name}[{b},{h}] pooled")
+
+
+@pytest.mark.parametrize("cfg", CASES, ids=lambda c: c.name)
+def test_spectral_norm_routing(lib, cfg):
+    q, k, v = inputs(cfg, redraws={})
+    qd, kd, vd = (to_device(x, cfg.dtype) for x in (q, k, v))
+    kk = lib.keep_count(cfg.L, cfg.block, cfg.keep_ratio)
+    stats = lib.block_stats(qd, kd, vd, cfg.block)
+    H = lib.block_first_order(kd, vd, cfg.block, stats[1], stats[2])
+    M = lib.cov_norm_spectral(H, stats[3], cfg.L, cfg.block)
+    sel = lib.select(stats[0], stats[1], M, cfg.L, cfg.block, kk)
+    torch.cuda.synchronize()
+    assert lib.device_status() == 0
+    s = 1.0 / math.sqrt(cfg.d)
+    for b in range(cfg.batch):
+        for h in range(cfg.heads):
+            r = oracle.pisa_head(q[b, h], k[b, h], v[b, h], cfg.block, kk, norm="spectral")
+            assert_stat_close(M[b, h].cpu().numpy(), r["M"], 1e-4, f"{cfg.name}[{b},{h}] spectral M")
+            assert (M[b, h].cpu().numpy() <= lib.cov_norm(kd, vd, cfg.block, stats[1], stats[2], stats[3])
+                    [b, h].cpu().numpy() * (1 + 1e-4)).all()
+            _compare_selection(sel[b, h].cpu().numpy(), r["scores"], kk, f"{cfg.name}[{b},{h}] spectral")
+            _check_output(lib, cfg, q, k, v, qd, kd, vd, stats, sel, b, h, f"{cfg.name}[{b},{h}] spectral")
+
+
+def test_spectral_norm_equals_frobenius_for_rank_one_deviations(lib):
+    """Keys c_j + a_n e (one direction, centred per block): every H_j - Hbar
+    has rank one, so its spectral and Frobenius norms coincide."""
+    L, B, d = 1024, 128, 128
+    rng = np.random.default_rng(61)
+    e = rng.standard_normal(d)
+    e /= np.linalg.norm(e)
+    a = rng.standard_normal(L)
+    for j in range(L // B):
+        a[j * B:(j + 1) * B] -= a[j * B:(j + 1) * B].mean()
+    k = rng.standard_normal((L // B, d))[np.arange(L) // B] + a[:, None] * e[None, :]
+    v = rng.standard_normal((L, d))
+    kd, vd = (torch.from_numpy(x.astype(np.float32)).cuda().reshape(1, 1, L, d) for x in (k, v))
+    stats = lib.block_stats(kd, kd, vd, B)
+    H = lib.block_first_order(kd, vd, B, stats[1], stats[2])
+    spec = lib.cov_norm_spectral(H, stats[3], L, B).cpu().numpy()
+    frob = lib.cov_norm(kd, vd, B, stats[1], stats[2], stats[3]).cpu().numpy()
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(spec, frob, rtol=1e-4)
