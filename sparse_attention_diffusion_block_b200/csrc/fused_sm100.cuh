@@ -516,12 +516,24 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
               }
               tmax = fmax3(fmaxf(t0, t1), t2, t3);
             } else {
+              // masked columns (an absent half, or past a ragged tail) become
+              // -inf; four independent three-input max chains
+              float t0 = -INFINITY, t1 = -INFINITY, t2 = -INFINITY, t3 = -INFINITY;
 #pragma unroll
-              for (int c = 0; c < 128; ++c) {
-                const float v = (c % KB) < nvalid[c / KB] ? __uint_as_float(s[c]) : -INFINITY;
-                s[c] = __float_as_uint(v);
-                tmax = fmaxf(tmax, v);
+              for (int c = 0; c < 128; c += 8) {
+                float v[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  const int cc = c + e;
+                  v[e] = (cc % KB) < nvalid[cc / KB] ? __uint_as_float(s[cc]) : -INFINITY;
+                  s[cc] = __float_as_uint(v[e]);
+                }
+                t0 = fmax3(t0, v[0], v[1]);
+                t1 = fmax3(t1, v[2], v[3]);
+                t2 = fmax3(t2, v[4], v[5]);
+                t3 = fmax3(t3, v[6], v[7]);
               }
+              tmax = fmax3(fmaxf(t0, t1), t2, t3);
             }
           } else {
             // centroid columns: masked when selected by this row's query block

@@ -47,10 +47,14 @@ bool all_ok(P... p) {
 }
 
 // Blocks per stats CTA: enough CTAs to fill the 148 SMs several times over
-// while keeping the partial-sum traffic (one d x d tile per CTA) small.
+// while keeping the partial-sum traffic (one d x d fp32 tile per CTA, written
+// and read back once) at most a third of the CTA's q, k, v reads (counted
+// for bf16): J >= 2 d / B.
 int stats_chunk(const Shape& s) {
   const long long target = 6LL * 148;
   long long J = ((long long)s.BH() * s.nb()) / target;
+  const long long jmin = (2LL * s.d + s.block - 1) / s.block;
+  if (J < jmin) J = jmin;
   if (J < 1) J = 1;
   if (J > s.nb()) J = s.nb();
   return (int)J;
