@@ -401,6 +401,8 @@ def main():
                     help="seconds of oracle time for the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--autotune", action="store_true",
+                    help="tune the result-invariant launch parameters for the workload first")
     ap.add_argument("--route", default="covariance", choices=["covariance", "pooled", "spectral"],
                     help="routing variant: the default covariance score with the Frobenius norm, "
                          "the pooled score, or the covariance score with the spectral norm")
@@ -482,6 +484,11 @@ def main():
         if ev: ev[3].record()
         pisa.attn_fwd_with_sel(qd, kd, vd, B, stats[1], stats[2], stats[3], sel, out=out, workspace=ws_fused)
         if ev: ev[4].record()
+
+    tuning = None
+    if args.autotune:
+        # result-invariant launch parameters, tuned once for this shape
+        tuning = pisa.autotune(qd, kd, vd, B, cfg.keep_ratio, out=out, workspace=ws_all)
 
     # correctness guard: the staged calls equal the one-shot entry point
     forward()
@@ -592,6 +599,7 @@ def main():
                        "seq_len": cfg.L, "parallelism": f"replicas x{world} (one full forward per GPU)",
                        "l2": f"inputs {3 * qd.numel() * qd.element_size() / 1e9:.2f} GB > L2 126 MB",
                        "route": args.route,
+                       "launch_tuning": tuning or "built-in heuristics",
                        "flops_exact": exact, "flops_approx": approx},
             "roofline": roofline,
             "stages": stages,

@@ -251,6 +251,43 @@ pisa_status pisa_attn_fwd_with_sel_noalloc(const void* q, const void* k, const v
                                            const float* hbar, const int32_t* sel, int k_sel,
                                            void* stream);
 
+/* Launch tuning.  A few launch parameters change only speed, never a
+ * result bit: the covariance-norm kernel's blocks per CTA (each M_j comes from
+ * its own block), the routing kernel's query blocks per CTA (rows are scored
+ * and selected independently) and the fused kernel's persistent CTA count
+ * (each pair of query tiles is computed by one CTA).  They are kept per
+ * (device, batch*heads, L, d, block); 0 in a field means the built-in
+ * heuristic.  Block size and the H-bar partial-sum grouping are not tuned:
+ * they would change results. */
+typedef struct pisa_tuning {
+  int cov_blocks_per_cta;   /* >= 0 */
+  int select_rows_per_cta;  /* 0..32, capped by shared memory */
+  int fused_ctas;           /* >= 0, capped by the SM count and the pairs of query tiles */
+} pisa_tuning;
+
+/* Times candidate values of each parameter on the given inputs (one
+ * parameter at a time, the others fixed; CUDA events on `stream`, three runs
+ * after a warm-up), keeps the fastest for this shape on the current device and
+ * returns it in `chosen` (may be NULL).  Blocking: synchronises `stream`.
+ * Runs the whole forward along the way: `out` receives its result.  Same
+ * arguments and workspace as pisa_attn_fwd. */
+pisa_status pisa_autotune(const void* q, const void* k, const void* v, void* out, pisa_dtype dtype,
+                          int batch, int heads, int L, int d, int block, float keep_ratio,
+                          void* workspace, size_t workspace_bytes, void* stream, pisa_tuning* chosen);
+
+/* Sets (t != NULL) or clears (t == NULL) the tuning of a shape on the current
+ * device; fields outside their ranges give PISA_ERR_INVALID_ARG. */
+pisa_status pisa_set_tuning(int batch, int heads, int L, int d, int block, const pisa_tuning* t);
+
+/* The tuning in force for a shape on the current device (all zero when none). */
+pisa_status pisa_get_tuning(int batch, int heads, int L, int d, int block, pisa_tuning* t);
+
+/* Writes the current device's tunings to a text file (one shape per line) /
+ * reads such a file into the current device's table.  A malformed file is
+ * rejected whole (PISA_ERR_INVALID_ARG) and changes nothing. */
+pisa_status pisa_tuning_save(const char* path);
+pisa_status pisa_tuning_load(const char* path);
+
 /* Reads (and, when reset != 0, clears) the device error word that bounded
  * waits and index checks set.  Synchronises `stream`.  Returns PISA_OK,
  * PISA_ERR_TIMEOUT, PISA_ERR_DEVICE_CHECK or PISA_ERR_CUDA. */

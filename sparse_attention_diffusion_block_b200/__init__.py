@@ -9,7 +9,8 @@ Entry points mirror the C names (without the ``pisa_`` prefix):
 block_stats, cov_norm, cov_norm_spectral, block_first_order, select, select_route,
 attn_fwd_with_sel, attn_fwd,
 attn_fwd_host, attn_fwd_with_sel_noalloc, keep_count, workspace_size, stats_workspace_size,
-fused_workspace_size, host_workspace_size, device_status, status_string.
+fused_workspace_size, host_workspace_size, autotune, set_tuning, clear_tuning, get_tuning,
+tuning_save, tuning_load, device_status, status_string.
 """
 
 from __future__ import annotations
@@ -48,7 +49,8 @@ EXPORTS = (
     "pisa_fused_workspace_size", "pisa_workspace_size", "pisa_block_stats", "pisa_cov_norm",
     "pisa_block_first_order", "pisa_select", "pisa_attn_fwd_with_sel", "pisa_attn_fwd",
     "pisa_device_status", "pisa_attn_fwd_with_sel_noalloc", "pisa_host_workspace_size",
-    "pisa_attn_fwd_host", "pisa_select_route", "pisa_cov_norm_spectral",
+    "pisa_attn_fwd_host", "pisa_select_route", "pisa_cov_norm_spectral", "pisa_autotune",
+    "pisa_set_tuning", "pisa_get_tuning", "pisa_tuning_save", "pisa_tuning_load",
 )
 
 _p = ctypes.c_void_p
@@ -83,6 +85,17 @@ _lib_device_status = _sig("pisa_device_status", _i, _p, _i)
 _lib_host_ws = _sig("pisa_host_workspace_size", _z, _i, _i, _i, _i, _i, _i, _i, _i)
 _lib_select_route = _sig("pisa_select_route", _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _p)
 _lib_cov_spectral = _sig("pisa_cov_norm_spectral", _i, _p, _p, _i, _i, _i, _i, _i, _p, _p)
+class _Tuning(ctypes.Structure):
+    _fields_ = [("cov_blocks_per_cta", ctypes.c_int), ("select_rows_per_cta", ctypes.c_int),
+                ("fused_ctas", ctypes.c_int)]
+
+
+_TP = ctypes.POINTER(_Tuning)
+_lib_autotune = _sig("pisa_autotune", _i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p, _z, _p, _TP)
+_lib_set_tuning = _sig("pisa_set_tuning", _i, _i, _i, _i, _i, _i, _TP)
+_lib_get_tuning = _sig("pisa_get_tuning", _i, _i, _i, _i, _i, _i, _TP)
+_lib_tuning_save = _sig("pisa_tuning_save", _i, ctypes.c_char_p)
+_lib_tuning_load = _sig("pisa_tuning_load", _i, ctypes.c_char_p)
 _lib_fwd_host = _sig("pisa_attn_fwd_host", _i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _i, _p, _z, _p)
 
 
@@ -293,6 +306,51 @@ def attn_fwd_host(q, k, v, block, keep_ratio, out=None, chunk=4, workspace=None,
                          float(keep_ratio), int(chunk), _ptr(ws), ws.numel(), _stream(stream)),
            "pisa_attn_fwd_host")
     return out
+
+
+def _tuning_dict(t: _Tuning) -> dict:
+    return {"cov_blocks_per_cta": t.cov_blocks_per_cta, "select_rows_per_cta": t.select_rows_per_cta,
+            "fused_ctas": t.fused_ctas}
+
+
+def autotune(q, k, v, block, keep_ratio, out=None, workspace=None, stream=None) -> dict:
+    """Times the result-invariant launch parameters for this shape on the
+    current device, keeps the fastest and returns them (blocking).  ``out``
+    receives the forward's result."""
+    _need_cuda(q, k, v)
+    b, h, L, d = _qkv_shape(q)
+    if out is None:
+        out = torch.empty_like(q)
+    kk = keep_count(L, block, keep_ratio)
+    ws = _workspace(workspace_size(b, h, L, d, block, kk), q.device, workspace)
+    t = _Tuning()
+    _check(_lib_autotune(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), b, h, L, d, block,
+                         float(keep_ratio), _ptr(ws), ws.numel(), _stream(stream), ctypes.byref(t)),
+           "pisa_autotune")
+    return _tuning_dict(t)
+
+
+def set_tuning(batch, heads, L, d, block, cov_blocks_per_cta=0, select_rows_per_cta=0, fused_ctas=0):
+    t = _Tuning(cov_blocks_per_cta, select_rows_per_cta, fused_ctas)
+    _check(_lib_set_tuning(batch, heads, L, d, block, ctypes.byref(t)), "pisa_set_tuning")
+
+
+def clear_tuning(batch, heads, L, d, block):
+    _check(_lib_set_tuning(batch, heads, L, d, block, None), "pisa_set_tuning")
+
+
+def get_tuning(batch, heads, L, d, block) -> dict:
+    t = _Tuning()
+    _check(_lib_get_tuning(batch, heads, L, d, block, ctypes.byref(t)), "pisa_get_tuning")
+    return _tuning_dict(t)
+
+
+def tuning_save(path: str):
+    _check(_lib_tuning_save(os.fsencode(path)), "pisa_tuning_save")
+
+
+def tuning_load(path: str):
+    _check(_lib_tuning_load(os.fsencode(path)), "pisa_tuning_load")
 
 
 def launches(entry: str, dtype: torch.dtype = torch.bfloat16) -> int:

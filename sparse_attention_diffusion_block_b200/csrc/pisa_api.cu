@@ -4,7 +4,9 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <tuple>
 #include <type_traits>
 
 #include "common.cuh"
@@ -28,6 +30,38 @@ struct Shape {
 };
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------------ launch tuning
+//
+// Launch parameters that cannot change any result, chosen per (device, shape)
+// by pisa_autotune or set explicitly; 0 means the built-in heuristic.
+//   cov_j:      blocks per CTA of the covariance-norm kernel (each M_j comes
+//               from its own block only)
+//   select_r:   query blocks per CTA of the routing kernel (rows are scored
+//               and selected independently)
+//   fused_ctas: persistent CTAs of the fused kernel (each pair of query tiles
+//               is computed by one CTA, whichever it is)
+struct Tuning {
+  int cov_j = 0, select_r = 0, fused_ctas = 0;
+};
+using TuneKey = std::tuple<int, int, int, int, int>;  // device, batch*heads, L, d, block
+std::mutex g_tune_mutex;
+std::map<TuneKey, Tuning> g_tune;
+
+bool tune_key(int bh, int L, int d, int block, TuneKey* key) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  *key = TuneKey{dev, bh, L, d, block};
+  return true;
+}
+
+Tuning tuning_for(int bh, int L, int d, int block) {
+  TuneKey key;
+  if (!tune_key(bh, L, d, block, &key)) return Tuning{};
+  std::lock_guard<std::mutex> lock(g_tune_mutex);
+  const auto it = g_tune.find(key);
+  return it == g_tune.end() ? Tuning{} : it->second;
+}
 
 pisa_status check_shape(const Shape& s) {
   if (s.batch < 1 || s.heads < 1 || s.L < 1 || s.d < 1 || s.block < 1) return PISA_ERR_INVALID_ARG;
@@ -156,6 +190,8 @@ pisa_status run_stats(const T* q, const T* k, const T* v, const Shape& s, float*
 }
 
 int cov_chunk(const Shape& s) {
+  const int tuned = tuning_for(s.BH(), s.L, s.d, s.block).cov_j;
+  if (tuned > 0) return tuned < s.nb() ? tuned : s.nb();
   long long J = ((long long)s.BH() * s.nb() + 8LL * 148 - 1) / (8LL * 148);
   if (J < 1) J = 1;
   if (J > s.nb()) J = s.nb();
@@ -190,18 +226,25 @@ pisa_status run_block_h(const T* k, const T* v, const Shape& s, const float* kba
   return last_launch();
 }
 
-int select_rows(int nb) {
+// Largest routing tile that fits: R rows of nb keys in 150 KB, at most 32.
+int select_rows_max(int nb) {
   const long long budget = 150 * 1024;
   long long R = budget / (4LL * nb);
   if (R > 32) R = 32;
   return (int)R;
 }
 
+int select_rows(const Shape& s) {
+  const int cap = select_rows_max(s.nb());
+  const int tuned = tuning_for(s.BH(), s.L, s.d, s.block).select_r;
+  return (tuned > 0 && tuned < cap) ? tuned : cap;
+}
+
 template <int D>
 pisa_status run_select(const float* qbar, const float* kbar, const float* M, const Shape& s, int k,
                        int32_t* sel, cudaStream_t st) {
   const int nb = s.nb();
-  const int R = select_rows(nb);
+  const int R = select_rows(s);
   if (R < 1) return PISA_ERR_UNSUPPORTED;
   const size_t smem = ((size_t)32 * D + 64 * (D + 4) + 32 + 128 + (size_t)R * nb) * sizeof(float);
   if (!set_smem(select_kernel<D>, smem)) return PISA_ERR_CUDA;
@@ -294,7 +337,9 @@ pisa_status run_fused_sm100(const __nv_bfloat16* q, const __nv_bfloat16* k, cons
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return PISA_ERR_CUDA;
-  const int grid = fa.n_pairs < sms ? fa.n_pairs : sms;
+  int grid = fa.n_pairs < sms ? fa.n_pairs : sms;
+  const int tuned = tuning_for(s.BH(), s.L, s.d, s.block).fused_ctas;
+  if (tuned > 0 && tuned < grid) grid = tuned;
   fused_sm100_kernel<D, KB><<<grid, kFusedThreads, smem, st>>>(mQ, mK, mV, mKc, mVc, mH, fa);
   return last_launch();
 }
@@ -508,6 +553,53 @@ pisa_status forward_host(const void* qh, const void* kh, const void* vh, void* o
     return PISA_ERR_CUDA;
   return PISA_OK;
 }
+// Mean time of `reps` runs of fn on st (after one warm-up run), in ms.
+template <typename F>
+pisa_status time_on(cudaStream_t st, int reps, F fn, float* ms) {
+  cudaEvent_t a, b;
+  if (cudaEventCreate(&a) != cudaSuccess) return PISA_ERR_CUDA;
+  if (cudaEventCreate(&b) != cudaSuccess) {
+    cudaEventDestroy(a);
+    return PISA_ERR_CUDA;
+  }
+  pisa_status e = fn();
+  if (!e && cudaEventRecord(a, st) != cudaSuccess) e = PISA_ERR_CUDA;
+  for (int r = 0; !e && r < reps; ++r) e = fn();
+  if (!e && (cudaEventRecord(b, st) != cudaSuccess || cudaEventSynchronize(b) != cudaSuccess ||
+             cudaEventElapsedTime(ms, a, b) != cudaSuccess))
+    e = PISA_ERR_CUDA;
+  if (!e) *ms /= reps;
+  cudaEventDestroy(a);
+  cudaEventDestroy(b);
+  return e;
+}
+
+void set_tuning(const TuneKey& key, const Tuning& t) {
+  std::lock_guard<std::mutex> lock(g_tune_mutex);
+  g_tune[key] = t;
+}
+
+// Tries each candidate of one parameter with the others fixed; keeps the fastest.
+template <typename F>
+pisa_status pick(const TuneKey& key, Tuning* t, int Tuning::*field, const int* cand, int n, cudaStream_t st,
+                 F run) {
+  float best_ms = 0.f;
+  int best = 0;
+  for (int c = 0; c < n; ++c) {
+    Tuning trial = *t;
+    trial.*field = cand[c];
+    set_tuning(key, trial);
+    float ms = 0.f;
+    if (pisa_status e = time_on(st, 3, run, &ms)) return e;
+    if (c == 0 || ms < best_ms) {
+      best_ms = ms;
+      best = cand[c];
+    }
+  }
+  t->*field = best;
+  set_tuning(key, *t);
+  return PISA_OK;
+}
 }  // namespace
 }  // namespace pisa
 
@@ -700,6 +792,136 @@ pisa_status pisa_attn_fwd_host(const void* q_host, const void* k_host, const voi
   if (!aligned16(workspace)) return PISA_ERR_INVALID_ARG;
   return forward_host(q_host, k_host, v_host, out_host, dtype, s, kk, hp, static_cast<char*>(workspace),
                       (cudaStream_t)stream);
+}
+
+pisa_status pisa_autotune(const void* q, const void* k, const void* v, void* out, pisa_dtype dtype, int batch,
+                          int heads, int L, int d, int block, float keep_ratio, void* workspace,
+                          size_t workspace_bytes, void* stream, pisa_tuning* chosen) {
+  const Shape s{batch, heads, L, d, block};
+  if (pisa_status e = check_shape(s)) return e;
+  if (!valid_dtype(dtype)) return PISA_ERR_INVALID_ARG;
+  const int kk = pisa_keep_count(L, block, keep_ratio);
+  if (kk < 1) return PISA_ERR_INVALID_ARG;
+  if (!all_ok(q, k, v, out)) return PISA_ERR_INVALID_ARG;
+  const Carve need = carve(s, kk, nullptr);
+  if (workspace == nullptr || workspace_bytes < need.total) return PISA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return PISA_ERR_INVALID_ARG;
+  TuneKey key;
+  if (!tune_key(s.BH(), L, d, block, &key)) return PISA_ERR_CUDA;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return PISA_ERR_CUDA;
+  const Carve c = carve(s, kk, static_cast<char*>(workspace));
+  cudaStream_t st = (cudaStream_t)stream;
+  Tuning t{};
+  set_tuning(key, t);
+  // inputs of the later stages: one default pass of stats and routing
+  pisa_status e = dispatch<StatsOp>(dtype, d, q, k, v, s, c.qbar, c.kbar, c.vsum, c.hbar, (float*)c.stats, st);
+  if (!e) e = dispatch<CovNormOp>(dtype, d, k, v, s, (const float*)c.kbar, (const float*)c.vsum,
+                                  (const float*)c.hbar, c.M, st);
+  if (!e) e = d == 128 ? run_select<128>(c.qbar, c.kbar, c.M, s, kk, c.sel, st)
+                       : run_select<64>(c.qbar, c.kbar, c.M, s, kk, c.sel, st);
+  if (e) return e;
+  // covariance norm: blocks per CTA around the heuristic
+  const int j0 = cov_chunk(s), nb = s.nb();
+  int cj[4] = {j0, j0 > 1 ? j0 / 2 : 1, j0 * 2 < nb ? j0 * 2 : nb, j0 * 4 < nb ? j0 * 4 : nb};
+  e = pick(key, &t, &Tuning::cov_j, cj, 4, st, [&] {
+    return dispatch<CovNormOp>(dtype, d, k, v, s, (const float*)c.kbar, (const float*)c.vsum,
+                               (const float*)c.hbar, c.M, st);
+  });
+  if (e) return e;
+  // routing: rows per CTA, up to what fits in shared memory
+  const int rmax = select_rows_max(nb);
+  int cr[4] = {rmax, rmax >= 24 ? 24 : rmax, rmax >= 16 ? 16 : rmax, rmax >= 8 ? 8 : rmax};
+  e = pick(key, &t, &Tuning::select_r, cr, 4, st, [&] {
+    return d == 128 ? run_select<128>(c.qbar, c.kbar, c.M, s, kk, c.sel, st)
+                    : run_select<64>(c.qbar, c.kbar, c.M, s, kk, c.sel, st);
+  });
+  if (e) return e;
+  // fused kernel: one CTA per SM, or the smallest grid with the same number of waves
+  const long long pairs = (long long)s.BH() * ((((long long)L + 127) / 128 + 1) / 2);
+  const long long waves = (pairs + sms - 1) / sms;
+  const int balanced = (int)((pairs + waves - 1) / waves);
+  int cf[3] = {sms, balanced < sms ? balanced : sms, sms - 4 > 0 ? sms - 4 : sms};
+  e = pick(key, &t, &Tuning::fused_ctas, cf, 3, st, [&] {
+    return dispatch<FusedOp>(dtype, d, q, k, v, out, s, (const float*)c.kbar, (const float*)c.vsum,
+                             (const float*)c.hbar, (const int32_t*)c.sel, kk, c.fused, st);
+  });
+  if (e) return e;
+  if (chosen) *chosen = pisa_tuning{t.cov_j, t.select_r, t.fused_ctas};
+  return PISA_OK;
+}
+
+pisa_status pisa_set_tuning(int batch, int heads, int L, int d, int block, const pisa_tuning* t) {
+  const Shape s{batch, heads, L, d, block};
+  if (pisa_status e = check_shape(s)) return e;
+  if (t && (t->cov_blocks_per_cta < 0 || t->select_rows_per_cta < 0 || t->select_rows_per_cta > 32 ||
+            t->fused_ctas < 0))
+    return PISA_ERR_INVALID_ARG;
+  TuneKey key;
+  if (!tune_key(s.BH(), L, d, block, &key)) return PISA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_tune_mutex);
+  if (t == nullptr) {
+    g_tune.erase(key);
+  } else {
+    g_tune[key] = Tuning{t->cov_blocks_per_cta, t->select_rows_per_cta, t->fused_ctas};
+  }
+  return PISA_OK;
+}
+
+pisa_status pisa_get_tuning(int batch, int heads, int L, int d, int block, pisa_tuning* t) {
+  const Shape s{batch, heads, L, d, block};
+  if (pisa_status e = check_shape(s)) return e;
+  if (t == nullptr) return PISA_ERR_INVALID_ARG;
+  const Tuning x = tuning_for(s.BH(), L, d, block);
+  *t = pisa_tuning{x.cov_j, x.select_r, x.fused_ctas};
+  return PISA_OK;
+}
+
+pisa_status pisa_tuning_save(const char* path) {
+  if (path == nullptr) return PISA_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PISA_ERR_CUDA;
+  FILE* f = std::fopen(path, "w");
+  if (f == nullptr) return PISA_ERR_INVALID_ARG;
+  std::fprintf(f, "# pisa launch tuning v1: batch*heads L d block cov_blocks_per_cta select_rows_per_cta fused_ctas\n");
+  {
+    std::lock_guard<std::mutex> lock(g_tune_mutex);
+    for (const auto& kv : g_tune) {
+      if (std::get<0>(kv.first) != dev) continue;
+      std::fprintf(f, "%d %d %d %d %d %d %d\n", std::get<1>(kv.first), std::get<2>(kv.first),
+                   std::get<3>(kv.first), std::get<4>(kv.first), kv.second.cov_j, kv.second.select_r,
+                   kv.second.fused_ctas);
+    }
+  }
+  return std::fclose(f) == 0 ? PISA_OK : PISA_ERR_INVALID_ARG;
+}
+
+pisa_status pisa_tuning_load(const char* path) {
+  if (path == nullptr) return PISA_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PISA_ERR_CUDA;
+  FILE* f = std::fopen(path, "r");
+  if (f == nullptr) return PISA_ERR_INVALID_ARG;
+  char line[256];
+  pisa_status status = PISA_OK;
+  std::map<TuneKey, Tuning> got;
+  while (std::fgets(line, sizeof line, f)) {
+    if (line[0] == '#' || line[0] == '\n') continue;
+    int bh, L, d, block, cj, sr, fc;
+    if (std::sscanf(line, "%d %d %d %d %d %d %d", &bh, &L, &d, &block, &cj, &sr, &fc) != 7 || bh < 1 ||
+        check_shape(Shape{1, bh, L, d, block}) != PISA_OK || cj < 0 || sr < 0 || sr > 32 || fc < 0) {
+      status = PISA_ERR_INVALID_ARG;
+      break;
+    }
+    got[TuneKey{dev, bh, L, d, block}] = Tuning{cj, sr, fc};
+  }
+  std::fclose(f);
+  if (status != PISA_OK) return status;  // a malformed file changes nothing
+  std::lock_guard<std::mutex> lock(g_tune_mutex);
+  for (const auto& kv : got) g_tune[kv.first] = kv.second;
+  return PISA_OK;
 }
 
 pisa_status pisa_device_status(void* stream, int reset) {

@@ -159,3 +159,22 @@ def test_routing_variant_entry_points_validate(lib):
     assert raw.pisa_cov_norm_spectral(FAKE, FAKE, 1, 1, 1000, 96, 128, FAKE, None) == lib.PISA_ERR_UNSUPPORTED
     assert raw.pisa_cov_norm_spectral(FAKE, FAKE, 1, 1, 1000, 128, 128, MISALIGNED, None) == \
         lib.PISA_ERR_INVALID_ARG
+
+
+def test_tuning_entry_points_validate_before_any_cuda_call(lib):
+    raw = lib.raw_lib()
+    t = lib._Tuning(0, 40, 0)  # select rows above 32
+    assert raw.pisa_set_tuning(1, 2, 1000, 128, 128, ctypes.byref(t)) == lib.PISA_ERR_INVALID_ARG
+    t = lib._Tuning(-1, 0, 0)
+    assert raw.pisa_set_tuning(1, 2, 1000, 128, 128, ctypes.byref(t)) == lib.PISA_ERR_INVALID_ARG
+    assert raw.pisa_set_tuning(1, 2, 1000, 96, 128, None) == lib.PISA_ERR_UNSUPPORTED
+    assert raw.pisa_get_tuning(1, 2, 1000, 128, 128, None) == lib.PISA_ERR_INVALID_ARG
+    assert raw.pisa_tuning_save(None) == lib.PISA_ERR_INVALID_ARG
+    assert raw.pisa_tuning_load(None) == lib.PISA_ERR_INVALID_ARG
+    f = raw.pisa_autotune
+    ok = [FAKE, FAKE, FAKE, FAKE, 0, 1, 2, 1000, 128, 128, ctypes.c_float(0.25), FAKE, ctypes.c_size_t(1 << 40),
+          None, None]
+    a = list(ok); a[3] = None
+    assert f(*a) == lib.PISA_ERR_INVALID_ARG                    # no output buffer
+    a = list(ok); a[12] = ctypes.c_size_t(64)
+    assert f(*a) == lib.PISA_ERR_WORKSPACE
