@@ -80,18 +80,37 @@ bool all_ok(P... p) {
   return true;
 }
 
-// Blocks per stats CTA: enough CTAs to fill the 148 SMs several times over
-// while keeping the partial-sum traffic (one d x d fp32 tile per CTA, written
-// and read back once) at most a third of the CTA's q, k, v reads (counted
-// for bf16): J >= 2 d / B.
+// Blocks per CTA for the two streaming kernels (one CTA per SM: they use
+// ~200 KB of shared memory).  A CTA's cost is its J blocks' input bytes plus a
+// fixed overhead (pipeline fill and drain, about three blocks' worth of
+// loads); the kernel's time follows the number of waves times that cost, so J
+// minimises ceil(CTAs / 148) x (J x block_bytes + extra).  The B200's 148 SMs
+// are a constant here so that workspace sizes do not depend on the device.
+constexpr int kSMs = 148;
+
+int wave_chunk(const Shape& s, long long block_bytes, long long extra, int jmin) {
+  const long long bh = s.BH(), nb = s.nb();
+  if (jmin < 1) jmin = 1;
+  if (jmin > nb) jmin = (int)nb;
+  long long best_cost = -1, best_j = jmin;
+  for (long long J = jmin; J <= nb; ++J) {
+    const long long ctas = bh * ((nb + J - 1) / J);
+    const long long waves = (ctas + kSMs - 1) / kSMs;
+    const long long cost = waves * (J * block_bytes + extra);
+    if (best_cost < 0 || cost < best_cost || (cost == best_cost && J > best_j)) {
+      best_cost = cost;
+      best_j = J;
+    }
+  }
+  return (int)best_j;
+}
+
+// Statistics kernel: reads q, k, v of each block (counted as bf16) and writes
+// one d x d fp32 partial of Hbar per CTA; at least 2d / B blocks per CTA keep
+// the partials under a third of the reads.
 int stats_chunk(const Shape& s) {
-  const long long target = 6LL * 148;
-  long long J = ((long long)s.BH() * s.nb()) / target;
-  const long long jmin = (2LL * s.d + s.block - 1) / s.block;
-  if (J < jmin) J = jmin;
-  if (J < 1) J = 1;
-  if (J > s.nb()) J = s.nb();
-  return (int)J;
+  const long long in = 3LL * s.block * s.d * 2, ovh = 3LL * in;
+  return wave_chunk(s, in, 4LL * s.d * s.d + ovh, (int)((2LL * s.d + s.block - 1) / s.block));
 }
 int stats_chunks(const Shape& s) {
   const int J = stats_chunk(s);
@@ -189,13 +208,12 @@ pisa_status run_stats(const T* q, const T* k, const T* v, const Shape& s, float*
   return last_launch();
 }
 
+// Covariance-norm kernel: reads k, v of each block; nothing per CTA but M.
 int cov_chunk(const Shape& s) {
   const int tuned = tuning_for(s.BH(), s.L, s.d, s.block).cov_j;
   if (tuned > 0) return tuned < s.nb() ? tuned : s.nb();
-  long long J = ((long long)s.BH() * s.nb() + 8LL * 148 - 1) / (8LL * 148);
-  if (J < 1) J = 1;
-  if (J > s.nb()) J = s.nb();
-  return (int)J;
+  const long long in = 2LL * s.block * s.d * 2;
+  return wave_chunk(s, in, 3LL * in, 1);
 }
 
 template <typename T, int D, bool WRITE_H>
