@@ -201,51 +201,83 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const int existsB = (tA + 1) < a.n_qtiles;
       for (int e = lane; e < 2 * G * words; e += 32) mA[e] = 0u;
       __syncwarp();
-      for (int x = 0; x < 1 + existsB; ++x) {
-        uint32_t* mX = x ? mB : mA;
-        for (int g = 0; g < G; ++g) {
-          const int i = (tA + x) * G + g;
-          if (i >= nb) continue;
-          const int32_t* si = a.sel + ((size_t)bh * nb + i) * a.kk;
-          for (int e = lane; e < a.kk; e += 32) {
-            const int j = si[e];
+      // Mask row r = x G + g is query block i = tA G + r; those rows are
+      // consecutive in sel, so the pair's selections are one flat run of
+      // n_sel entries.  Loads go out eight per lane before any atomic, so the
+      // run costs a couple of L2 round trips, not one per 32 entries.
+      {
+        const int rows = min((1 + existsB) * G, nb - tA * G);
+        const int n_sel = rows * a.kk;
+        const int32_t* run = a.sel + ((size_t)bh * nb + (size_t)tA * G) * a.kk;
+        for (int e0 = 0; e0 < n_sel; e0 += 32 * 8) {
+          int jv[8];
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const int e = e0 + lane + 32 * m;
+            jv[m] = e < n_sel ? __ldg(run + e) : 0;
+          }
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const int e = e0 + lane + 32 * m;
+            if (e >= n_sel) continue;
+            const int j = jv[m];
             if (j < 0 || j >= nb) {
               raise_device_error(PISA_ERR_DEVICE_CHECK);
             } else {
-              atomicOr(&mX[g * words + (j >> 5)], 1u << (j & 31));
+              atomicOr(&mA[(e / a.kk) * words + (j >> 5)], 1u << (j & 31));
             }
           }
         }
       }
       __syncwarp();
-      if (lane == 0) {
-        int nA = 0, nB = 0, nC = 0;
-        // pass 0: blocks of both tiles; pass 1: A only; pass 2: B only
-        for (int pass = 0; pass < 3; ++pass) {
-          for (int w = 0; w < words; ++w) {
+      // Entry lists, all lanes: pass 0 the blocks of both tiles, pass 1 of A
+      // only, pass 2 of B only, each ascending.  Lane l owns mask word w0 + l;
+      // a warp scan of the words' bit counts gives each lane its output slot.
+      int nA = 0, nB = 0, nC = 0;
+      for (int pass = 0; pass < 3; ++pass) {
+        for (int w0 = 0; w0 < words; w0 += 32) {
+          const int w = w0 + lane;
+          uint32_t bits = 0u;
+          if (w < words) {
             uint32_t uA = 0, uB = 0;
 #pragma unroll
             for (int g = 0; g < G; ++g) {
               uA |= mA[g * words + w];
               uB |= mB[g * words + w];
             }
-            uint32_t bits = pass == 0 ? (uA & uB) : pass == 1 ? (uA & ~uB) : (uB & ~uA);
-            while (bits) {
-              const int b = __ffs(bits) - 1;
-              bits &= bits - 1;
-              int gA = 0, gB = 0;
-#pragma unroll
-              for (int g = 0; g < G; ++g) {
-                gA |= ((mA[g * words + w] >> b) & 1u) << g;
-                gB |= ((mB[g * words + w] >> b) & 1u) << g;
-              }
-              const int j = w * 32 + b;
-              if (pass != 2) eA[nA++] = j | (gA << 24);
-              if (pass != 1) eB[nB++] = j | (gB << 24);
-              if (pass == 0) ++nC;
-            }
+            bits = pass == 0 ? (uA & uB) : pass == 1 ? (uA & ~uB) : (uB & ~uA);
           }
+          const int c = __popc(bits);
+          int incl = c;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+          }
+          const int total = __shfl_sync(0xffffffffu, incl, 31);
+          int pos = (pass == 2 ? nB : nA) + incl - c;
+          while (bits) {
+            const int b = __ffs(bits) - 1;
+            bits &= bits - 1;
+            int gA = 0, gB = 0;
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+              gA |= ((mA[g * words + w] >> b) & 1u) << g;
+              gB |= ((mB[g * words + w] >> b) & 1u) << g;
+            }
+            const int j = w * 32 + b;
+            if (pass != 2) eA[pos] = j | (gA << 24);
+            if (pass != 1) eB[pos] = j | (gB << 24);
+            ++pos;
+          }
+          if (pass != 2) nA += total;
+          if (pass != 1) nB += total;
+          if (pass == 0) nC += total;
         }
+      }
+      __threadfence_block();
+      __syncwarp();
+      if (lane == 0) {
         // header: steps of A, B and shared steps (a step = 128 keys: one 128-token
         // block, or two consecutive list entries of 64 tokens), then the entry counts
         L_[0] = (nA + G - 1) / G;
@@ -374,42 +406,59 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         fence_after_sync();
         int ks = -1, vs = -1;  // slots of the last K / V items
         bool first_pv[2] = {true, true};
-        auto issue_s = [&](int x, int u) -> bool {
+        auto s_mmas = [&](int x) {
           const uint32_t sc = tmem + x * 128;
-          if (!((x == 1) && pl.shared(u)) && !take(ks)) return false;  // tile B reuses tile A's items when shared
           for (int kk = 0; kk < D / 16; ++kk) mma_ss_warp(sc, qdesc(x, kk), kdesc(ks, 128, kk), idC, kk > 0 ? 1u : 0u);
-          if (!((x == 0) && pl.shared(u))) mma_commit_warp(&empty[ks]);
+        };
+        // Step u of tile x: O_x += P_x(u) V(u), then S_x = Q_x K(u+1)^T.  Both
+        // ring items are taken before the wait for P, so their barrier waits
+        // overlap the softmax instead of sitting between P and the next S; the
+        // two MMA groups go out back to back and the commits follow them.  The
+        // tensor pipe runs a CTA's MMAs in issue order, so S(u+1) overwrites
+        // the S/P columns only after PV(u) has read P(u).
+        auto issue_step = [&](int x, int u) -> bool {
+          const bool pv = x == 0 ? pl.activeA(u) : pl.activeB(u);
+          const bool sn = u + 1 < T && (x == 0 ? pl.activeA(u + 1) : pl.activeB(u + 1));
+          // tile B reuses tile A's items on shared steps; tile A then keeps them
+          if (pv && !((x == 1) && pl.shared(u)) && !take(vs)) return false;
+          if (sn && !((x == 1) && pl.shared(u + 1)) && !take(ks)) return false;
+          if (pv) {
+            if (!mbar_wait(&p_full[x], steps[x] & 1, abort)) return false;
+            ++steps[x];
+            fence_after_sync();
+            const uint32_t pa = tmem + x * 128;
+            const uint32_t oc = tmem + OC + x * D;
+            // one V item per step: a 128-token value tile or 128 centroid value sums
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ts_warp(oc, pa + kk * 8, vdesc(vs, 128, kk), idO, (!first_pv[x] || kk > 0) ? 1u : 0u);
+            first_pv[x] = false;
+          }
+          if (sn) s_mmas(x);
+          if (pv && !((x == 0) && pl.shared(u))) mma_commit_warp(&empty[vs]);
+          if (sn) {
+            if (!((x == 0) && pl.shared(u + 1))) mma_commit_warp(&empty[ks]);
+            mma_commit_warp(&s_full[x]);
+          }
+          return true;
+        };
+        // first S of a tile: before reusing S_x / O_x the previous epilogue of
+        // tile x must have read them
+        auto issue_first_s = [&](int x) -> bool {
+          if (epis[x] > 0) {
+            if (!mbar_wait(&epi_done[x], (epis[x] - 1) & 1, abort)) return false;
+            fence_after_sync();
+          }
+          if (!((x == 1) && pl.shared(0)) && !take(ks)) return false;
+          s_mmas(x);
+          if (!((x == 0) && pl.shared(0))) mma_commit_warp(&empty[ks]);
           mma_commit_warp(&s_full[x]);
           return true;
         };
-        auto issue_pv = [&](int x, int u) -> bool {
-          if (!mbar_wait(&p_full[x], steps[x] & 1, abort)) return false;
-          ++steps[x];
-          fence_after_sync();
-          const uint32_t pa = tmem + x * 128;
-          const uint32_t oc = tmem + OC + x * D;
-          // one V item per step: a 128-token value tile or 128 centroid value sums
-          if (!((x == 1) && pl.shared(u)) && !take(vs)) return false;
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts_warp(oc, pa + kk * 8, vdesc(vs, 128, kk), idO, (!first_pv[x] || kk > 0) ? 1u : 0u);
-          first_pv[x] = false;
-          if (!((x == 0) && pl.shared(u))) mma_commit_warp(&empty[vs]);
-          return true;
-        };
-        // before reusing S_x / O_x the previous epilogue of tile x must have read them
-        auto epi_wait = [&](int x) -> bool {
-          if (epis[x] == 0) return true;
-          if (!mbar_wait(&epi_done[x], (epis[x] - 1) & 1, abort)) return false;
-          fence_after_sync();
-          return true;
-        };
-        ok = epi_wait(0) && issue_s(0, 0);
-        if (ok && pl.activeB(0)) ok = epi_wait(1) && issue_s(1, 0);
+        ok = issue_first_s(0);
+        if (ok && pl.activeB(0)) ok = issue_first_s(1);
         for (int u = 0; ok && u < T; ++u) {
-          if (pl.activeA(u)) ok = issue_pv(0, u);
-          if (ok && u + 1 < T && pl.activeA(u + 1)) ok = issue_s(0, u + 1);
-          if (ok && pl.activeB(u)) ok = issue_pv(1, u);
-          if (ok && u + 1 < T && pl.activeB(u + 1)) ok = issue_s(1, u + 1);
+          ok = issue_step(0, u);
+          if (ok && pl.existsB) ok = issue_step(1, u);
         }
         if (!ok) break;
         // first-order term q Hbar into each tile's S columns; then Q and Hbar are free
