@@ -517,31 +517,22 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         uint32_t s[128];
         for (int u = 0; u < T; ++u) {
           if (!(x == 0 ? pl.activeA(u) : pl.activeB(u))) continue;
-          if (!__all_sync(0xffffffffu, mbar_wait(&s_full[x], steps & 1, abort))) {
-            ok = false;
-            break;
-          }
-          ++steps;
-          fence_after_sync();
           const bool exact = !pl.centroid(u);
-          float tmax = -INFINITY, x_tail = -INFINITY;
-          tmem_ld32(sbase, s);
-          tmem_ld32(sbase + 32, s + 32);
-          tmem_ld32(sbase + 64, s + 64);
-          tmem_ld32(sbase + 96, s + 96);
-          tmem_wait_ld();
+          // Which keys of an exact step this row may use depends only on the
+          // work list, so it is settled before the wait for S.  Column half h
+          // (of KB columns) holds list entry G u + h: all of its tokens count if
+          // the row's query block selected it, none otherwise (or when the
+          // entry is absent).  The tile's list entries sit in a 32-entry
+          // register window, one per lane, refilled every 32 entries.
+          int nvalid[G];
+          bool all_whole = false;
           if (exact) {
-            // column half h (of KB columns) holds list entry G u + h; the keys of
-            // that block this row may use: all of its tokens if the row's query
-            // block selected it, none otherwise (or when the entry is absent)
-            // the tile's list entries sit in a 32-entry register window, one
-            // per lane, refilled from shared memory every 32 entries
             if (((G * u) >> 5) != ent_win) {
               ent_win = (G * u) >> 5;
               const int idx = ent_win * 32 + lane;
               ent_reg = idx < n_ent ? ent[idx] : 0;
             }
-            int nvalid[G];
+            bool whole = true;
 #pragma unroll
             for (int h = 0; h < G; ++h) {
               nvalid[h] = 0;
@@ -550,11 +541,24 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 const int j = e & 0xFFFFFF;
                 if ((e >> (24 + g)) & 1) nvalid[h] = min(KB, a.L - j * KB);
               }
+              whole = whole && nvalid[h] == KB;
             }
-            bool whole = true;
-#pragma unroll
-            for (int h = 0; h < G; ++h) whole = whole && nvalid[h] == KB;
-            if (__all_sync(0xffffffffu, whole)) {
+            all_whole = __all_sync(0xffffffffu, whole);
+          }
+          if (!__all_sync(0xffffffffu, mbar_wait(&s_full[x], steps & 1, abort))) {
+            ok = false;
+            break;
+          }
+          ++steps;
+          fence_after_sync();
+          float tmax = -INFINITY, x_tail = -INFINITY;
+          tmem_ld32(sbase, s);
+          tmem_ld32(sbase + 32, s + 32);
+          tmem_ld32(sbase + 64, s + 64);
+          tmem_ld32(sbase + 96, s + 96);
+          tmem_wait_ld();
+          if (exact) {
+            if (all_whole) {
               float t0 = -INFINITY, t1 = -INFINITY, t2 = -INFINITY, t3 = -INFINITY;
 #pragma unroll
               for (int c = 0; c < 128; c += 8) {
@@ -650,6 +654,7 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             const float p1 = ex2(f2_hi(t));
             acc = fadd2(acc, f2_pack(p0, p1));
             s[c >> 1] = pack_bf16x2(p0, p1);
+            if (c == 62) tmem_st32(sbase, s);  // keys 0..63 go out while 64..127 are computed
           }
           const float sum = f2_lo(acc) + f2_hi(acc);
           if (exact) {
@@ -659,7 +664,6 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             l += (float)a.block * sum;
             if (x_tail != -INFINITY) l += (float)(n_tail - a.block) * ex2(x_tail * c2 - mu);
           }
-          tmem_st32(sbase, s);
           tmem_st32(sbase + 32, s + 32);
           tmem_wait_st();
           fence_before_sync();
