@@ -17,14 +17,19 @@
 //              rescales O in TMEM when m grows by more than 8 (log2 units;
 //              exact since N and D carry the same factor), epilogue
 //              o = (O + s beta q Hbar) / l.
-//   warp 8     producer: builds each pair's work list in shared memory, then
-//              streams Q tiles and a ring of 128-row operand tiles with TMA.
+//   warp 8     producer: streams Q tiles and a ring of 128-row operand tiles
+//              with TMA, in the order of each pair's work list.
 //   warp 9     MMA issuer: S = Q K^T and O += P V (P from TMEM), ping-ponging
 //              the two tiles so that one tile's softmax overlaps the other
 //              tile's MMAs.  The whole warp runs the issue loop and one
 //              elected lane issues each instruction, which keeps the operands
 //              in warp-uniform registers (a lone lane in a divergent branch
-//              issues markedly slower).
+//              issues markedly slower).  Each step's ring items are taken
+//              before the wait for P, and the PV and next-S groups go out back
+//              to back.
+//   warp 10    list builder: builds each pair's work list in shared memory
+//              (two slots) one pair ahead of the other roles.
+//   warp 11    idle.
 // Work list of a pair: the exact KV blocks of each tile (for 64-token blocks a
 // 128-row tile spans two query blocks: the union, with per-row-group bits),
 // blocks selected by both tiles first and in the same order, so those K/V
@@ -151,7 +156,7 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       mbar_init(&o_final[x], 1);
       mbar_init(&epi_done[x], 128);
       mbar_init(&list_full[x], 1);
-      mbar_init(&list_empty[x], 9);
+      mbar_init(&list_empty[x], 10);
     }
     mbar_init(mma_idle, 1);
     *abort = 0;
@@ -172,17 +177,11 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   // launch total would wait forever).
   if (warp >= 8) {
    asm volatile("setmaxnreg.dec.sync.aligned.u32 104;\n" ::: "memory");
-   if (warp == 8) {
-    // ================================================================ producer
-    if (lane == 0) {
-      prefetch_tensormap(&tmQ);
-      prefetch_tensormap(&tmK);
-      prefetch_tensormap(&tmV);
-      prefetch_tensormap(&tmKc);
-      prefetch_tensormap(&tmVc);
-      prefetch_tensormap(&tmH);
-    }
-    int it = 0, qloads[2] = {0, 0};
+   if (warp == 10) {
+    // ============================================================ list builder
+    // Builds each pair's work list (header, entry lists, selection masks) one
+    // pair ahead of the producer, the MMA issuer and the softmax warps, so that
+    // none of them waits for it between pairs.
     bool ok = true;
     int lp = 0;
     for (int p = blockIdx.x; ok && p < a.n_pairs; p += gridDim.x, ++lp) {
@@ -298,8 +297,36 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           }
         }
         mbar_arrive(&list_full[slot]);
-
-        const PairPlan pl{(nA + G - 1) / G, (nB + G - 1) / G, nC / G, existsB, n_cent};
+      }
+    }
+   } else if (warp == 8) {
+    // ================================================================ producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmQ);
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      prefetch_tensormap(&tmKc);
+      prefetch_tensormap(&tmVc);
+      prefetch_tensormap(&tmH);
+    }
+    int it = 0, qloads[2] = {0, 0};
+    bool ok = true;
+    int lp = 0;
+    for (int p = blockIdx.x; ok && p < a.n_pairs; p += gridDim.x, ++lp) {
+      const int slot = lp & 1;
+      const int* L_ = lists + slot * list_stride;
+      const int* eA = L_ + 8;
+      const int* eB = eA + G * a.kk;
+      if (!__all_sync(0xffffffffu, mbar_wait(&list_full[slot], (lp >> 1) & 1, abort))) {
+        ok = false;
+        break;
+      }
+      const int bh = p / pairs_per_head;
+      const int tA = 2 * (p % pairs_per_head);
+      const int existsB = (tA + 1) < a.n_qtiles;
+      if (lane == 0) {
+        const int nA = L_[6], nB = L_[7];  // entry counts
+        const PairPlan pl{L_[0], L_[1], L_[2], L_[3], n_cent};
         // one ring item: `rows` rows at `row`, and when row2 >= 0 another `rows`
         // rows at row2 stacked below them (a 2 x 64-row step)
         auto load = [&](const CUtensorMap* map, int row, int rows, int row2) -> bool {
@@ -353,6 +380,8 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           if (ok && u + 1 < T && pl.activeB(u + 1) && !pl.shared(u + 1)) ok = loadK(1, u + 1);
         }
         if (ok) ok = load(&tmH, 0, D, -1) && load(&tmH, D, D, -1);
+        // every copy of the pair is issued: the list is no longer read here
+        if (ok) mbar_arrive(&list_empty[slot]);
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     }
