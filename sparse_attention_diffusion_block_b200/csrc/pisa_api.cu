@@ -246,7 +246,8 @@ pisa_status run_block_h(const T* k, const T* v, const Shape& s, const float* kba
 
 // Largest routing tile that fits: R rows of nb keys in 150 KB, at most 32.
 int select_rows_max(int nb) {
-  const long long budget = 150 * 1024;
+  // the key buffer (R x nb words) beside the fixed tiles, within 227 KB
+  const long long budget = 140 * 1024;
   long long R = budget / (4LL * nb);
   if (R > 32) R = 32;
   return (int)R;
@@ -264,10 +265,10 @@ pisa_status run_select(const float* qbar, const float* kbar, const float* M, con
   const int nb = s.nb();
   const int R = select_rows(s);
   if (R < 1) return PISA_ERR_UNSUPPORTED;
-  const size_t smem = ((size_t)32 * D + 64 * (D + 4) + 32 + 128 + (size_t)R * nb) * sizeof(float);
+  const size_t smem = select_smem_bytes(D, R, nb);
   if (!set_smem(select_kernel<D>, smem)) return PISA_ERR_CUDA;
   const float scale = 1.0f / sqrtf((float)D);
-  select_kernel<D><<<dim3((nb + R - 1) / R, s.BH()), 256, smem, st>>>(qbar, kbar, M, s.L, s.block, nb,
+  select_kernel<D><<<dim3((nb + R - 1) / R, s.BH()), kSelectThreads, smem, st>>>(qbar, kbar, M, s.L, s.block, nb,
                                                                       k, R, scale, sel);
   return last_launch();
 }

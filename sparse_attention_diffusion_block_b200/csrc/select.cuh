@@ -17,22 +17,33 @@ __device__ __forceinline__ uint32_t orderable_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Grid (ceil(nb / R), BH), 256 threads (8 warps), R <= 32, dynamic smem:
-//   Qb [32][D] fp32 (rows >= R zero), Kc [64][D+4] fp32, qn [32], mj [64],
-//   nj [64], keys [R][nb] uint32.
-// Phase 1 computes the R x nb scores with fp32 FMAs, 64 key blocks at a time,
-// each thread a 2 x 4 register tile (rows tr, tr+16; key columns tc + 16c), and
-// stores their orderable keys; phase 2 runs, per row (one warp per row), an
+constexpr int kSelectThreads = 512;  // 16 warps
+constexpr int kSelectKT = 128;       // key blocks per score tile
+
+// Shared memory of select_kernel<D> for R query blocks per CTA.
+__host__ __device__ constexpr size_t select_smem_bytes(int D, int R, int nb) {
+  return ((size_t)32 * D + (size_t)kSelectKT * (D + 4) + 32 + 2 * kSelectKT + (size_t)R * nb) * sizeof(float);
+}
+
+// Grid (ceil(nb / R), BH), kSelectThreads threads, R <= 32, dynamic smem:
+//   Qb [32][D] fp32 (rows >= R zero), Kc [KT][D+4] fp32, qn [32], mj [KT],
+//   nj [KT], keys [R][nb] uint32.
+// Phase 1 computes the R x nb scores with fp32 FMAs, KT key blocks at a time;
+// each thread holds a 2 x 4 register tile (rows tr, tr+16; key columns
+// 64 h + tc + 16c, h the thread's half of the CTA), and stores their orderable
+// keys.  The CTA's sixteen warps keep the latency-bound score and selection
+// loops busy at one CTA per SM.  Phase 2 runs, per row (one warp per row), an
 // MSB-first bitwise search for the k-th largest key, then writes the selected
 // indices in ascending order.
 template <int D>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kSelectThreads)
 select_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
               const float* __restrict__ M, int L, int B, int nb, int kk, int R,
               float scale, int32_t* __restrict__ sel) {
   extern __shared__ __align__(16) float sm[];
   constexpr int KS = D + 4;
-  constexpr int KT = 64;                       // key blocks per tile
+  constexpr int KT = kSelectKT;                // key blocks per tile
+  constexpr int NW = kSelectThreads / 32;      // warps
   float* Qb = sm;                              // 32 * D
   float* Kc = Qb + 32 * D;                     // KT * KS
   float* qn = Kc + KT * KS;                    // 32
@@ -49,7 +60,7 @@ select_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
     Qb[e] = (r < rows) ? qbar[((size_t)bh * nb + i0 + r) * D + (e % D)] : 0.f;
   }
   __syncthreads();
-  for (int r = warp; r < 32; r += 8) {
+  for (int r = warp; r < 32; r += NW) {
     float t = 0.f;
     for (int a = lane; a < D; a += 32) t = fmaf(Qb[r * D + a], Qb[r * D + a], t);
     t = warp_sum(t);
@@ -57,7 +68,7 @@ select_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
   }
 
   // Phase 1: scores.
-  const int tr = threadIdx.x >> 4, tc = threadIdx.x & 15;
+  const int tr = (threadIdx.x & 255) >> 4, tc = threadIdx.x & 15, ch = (threadIdx.x >> 8) * 64;
   for (int j0 = 0; j0 < nb; j0 += KT) {
     __syncthreads();
     for (int e = threadIdx.x; e < KT * (D / 4); e += blockDim.x) {
@@ -83,7 +94,7 @@ select_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
       const float4 q1 = *reinterpret_cast<const float4*>(Qb + (tr + 16) * D + a);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const float4 k = *reinterpret_cast<const float4*>(Kc + (tc + 16 * c) * KS + a);
+        const float4 k = *reinterpret_cast<const float4*>(Kc + (ch + tc + 16 * c) * KS + a);
         acc[0][c] = fmaf(q0.x, k.x, acc[0][c]);
         acc[0][c] = fmaf(q0.y, k.y, acc[0][c]);
         acc[0][c] = fmaf(q0.z, k.z, acc[0][c]);
@@ -100,7 +111,7 @@ select_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
       if (r >= rows) continue;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const int cl = tc + 16 * c;
+        const int cl = ch + tc + 16 * c;
         const int j = j0 + cl;
         if (j < nb) keys[r * nb + j] = orderable_key(scale * acc[rr][c] + logf(nj[cl] + scale * qn[r] * mj[cl]));
       }
@@ -110,7 +121,7 @@ select_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
 
   // Phase 2: per-row selection.
   const int C = (nb + 31) / 32;  // contiguous chunk of indices per lane
-  for (int r = warp; r < rows; r += 8) {
+  for (int r = warp; r < rows; r += NW) {
     const uint32_t* kr = keys + r * nb;
     uint32_t thr;  // k-th largest key
     if (nb <= 1024) {
