@@ -31,10 +31,13 @@ spectral norm for M_j (R6), the pooled score without the covariance term
 (R7), and the un-hybridised first-order term with each unselected block's own
 H_j (the summary's starting point before Hbar).
 
-Parity unpinned: the routing score formula (R7) and the norm choice (R6).
-Nothing on the pages fixes them; the tests pin their structure (V = 0 reduces
-the score to pooled block-sparse routing; permutation invariance) but not the
-formula itself.
+The pages print neither the routing score nor the matrix norm, so R6 and R7
+are readings, not formulas taken from the pages.  Each function that
+implements them is pinned to the reading's own derivation: the score equals
+the log of alpha n_j plus the first-order error bound alpha ||s qbar_i (H_j -
+Hbar)|| wherever Cauchy-Schwarz is tight (rank-one deviations with qbar_i
+parallel to them), the ranking is monotone in M_j at equal centroids, V = 0
+reduces it to pooled block-sparse routing, and M_j meets closed forms.
 """
 
 from .pisa_ref import (  # noqa: F401

@@ -100,7 +100,7 @@ def hbar_mean(H: np.ndarray) -> np.ndarray:
 
 def cov_norm(H: np.ndarray, Hbar: np.ndarray) -> np.ndarray:
     """M_j = ||H_j - Hbar|| (gist.science summary, section 2, covariance-aware
-    routing), with the Frobenius norm (reading R6; parity unpinned)."""
+    routing), with the Frobenius norm (reading R6)."""
     diff = H - Hbar[None, :, :]
     return np.sqrt((diff * diff).sum(axis=(1, 2)))
 
@@ -124,7 +124,7 @@ def route_scores_pooled(qbar: np.ndarray, kbar: np.ndarray, n: np.ndarray, s: fl
 
 
 def route_scores(qbar: np.ndarray, kbar: np.ndarray, M: np.ndarray, n: np.ndarray, s: float) -> np.ndarray:
-    """Routing score of KV block j for query block i (reading R7; parity unpinned).
+    """Routing score of KV block j for query block i (reading R7).
 
     score_{i,j} = s qbar_i . kbar_j + ln(n_j + s ||qbar_i||_2 M_j): the log of
     the block's zeroth-order softmax mass times (its size plus the

@@ -294,6 +294,105 @@ def test_scores_reduce_to_pooled_when_covariance_norm_constant():
     np.testing.assert_array_equal(oracle.select_topk(a, 3), oracle.select_topk(b, 3))
 
 
+def _aligned_rank_one_case(L=230, B=20, d=8, seed=41):
+    """Raw Q, K, V whose block statistics are known in closed form.
+
+    Keys k_n = c_j + a_n e (unit direction e, per-block centred scalars a_n),
+    so kbar_j = c_j and H_j - Hbar = e (w_j - wbar)^T with w_j = sum_n a_n v_n
+    (rank one).  Queries q_t = b_i e + r_t with per-block centred noise r_t,
+    so qbar_i = b_i e is parallel to e.  The last block is partial (L is not
+    a multiple of B), so n_j is not constant.  Returns q, k, v and the closed
+    forms (b, c, w, n)."""
+    rng = np.random.default_rng(seed)
+    nb = -(-L // B)
+    blk = np.arange(L) // B
+    e = rng.standard_normal(d)
+    e /= np.linalg.norm(e)
+
+    def centred(x):
+        x = x.copy()
+        for j in range(nb):
+            x[blk == j] -= x[blk == j].mean(axis=0)
+        return x
+
+    a = centred(rng.standard_normal(L))
+    c = rng.standard_normal((nb, d))
+    k = c[blk] + a[:, None] * e[None, :]
+    v = rng.standard_normal((L, d))
+    # |b_i| spread well away from 1, so a squared norm cannot pass for the norm
+    b = rng.choice([-1.0, 1.0], nb) * rng.uniform(0.3, 3.0, nb)
+    q = b[blk][:, None] * e[None, :] + centred(rng.standard_normal((L, d)))
+    w = np.stack([(a[blk == j, None] * v[blk == j]).sum(axis=0) for j in range(nb)])
+    n = np.bincount(blk).astype(np.float64)
+    return q, k, v, (b, c, e, w, n)
+
+
+def test_routing_score_is_the_tight_cauchy_schwarz_bound_on_rank_one_blocks():
+    """Score_{i,j} (reading R7) from raw inputs, without the oracle's norm.
+
+    The score is the log of block j's zeroth-order softmax mass alpha n_j plus
+    the bound alpha ||s qbar_i (H_j - Hbar)|| on the first-order error that
+    Hbar leaves in that block (gist.science summary, section 2,
+    covariance-aware routing; AI Radio summary, Score_{t,j}).  When H_j - Hbar
+    = e u_j^T and qbar_i is parallel to e, Cauchy-Schwarz is an equality:
+    ||s qbar_i (H_j - Hbar)|| = s ||qbar_i|| ||H_j - Hbar||, so the score must
+    equal ln(alpha_ij n_j + ||alpha_ij s qbar_i (H_j - Hbar)||) with
+    alpha_ij = exp(s qbar_i . kbar_j), every factor taken from the
+    construction.  A dropped s, a squared query norm, or the log split as
+    ln n_j + s||qbar||M_j each fail this."""
+    L, B, d = 230, 20, 8
+    q, k, v, (b, c, e, w, n) = _aligned_rank_one_case(L, B, d)
+    s = 1.0 / math.sqrt(d)
+    r = oracle.pisa_head(q, k, v, B, 3)
+    np.testing.assert_allclose(r["kbar"], c, atol=1e-12)
+    np.testing.assert_allclose(r["qbar"], b[:, None] * e[None, :], atol=1e-12)
+    u = w - w.mean(axis=0)  # H_j - Hbar = e u_j^T
+    qbar = b[:, None] * e[None, :]
+    for i in range(len(b)):
+        for j in range(len(n)):
+            alpha = math.exp(s * float(qbar[i] @ c[j]))
+            err_vec = s * (qbar[i] @ np.outer(e, u[j]))  # s qbar_i (H_j - Hbar), a d-vector
+            want = math.log(alpha * n[j] + alpha * float(np.linalg.norm(err_vec)))
+            assert abs(r["scores"][i, j] - want) <= 1e-12 * max(1.0, abs(want)), (i, j)
+    # the construction really exercises the covariance term: it moves the
+    # scores by far more than the tolerance, and n_j differs on the tail
+    assert np.abs(r["scores"] - (s * qbar @ c.T + np.log(n)[None, :])).max() > 0.1
+    assert n[-1] != n[0]
+
+
+def test_routing_ranks_blocks_by_covariance_norm_at_equal_centroids():
+    """Monotone in M_j: blocks with the same centroid and size differ only in
+    their covariance norm, and for any query block with qbar_i != 0 the block
+    with the larger M_j scores higher (the error bound grows with it).
+
+    Block j's keys are the centroid plus a shared centred pattern scaled by
+    t_j = 2^j, with the same values in every block, so H_j = t_j H_0, Hbar =
+    mean(t) H_0 and M_j = |t_j - mean(t)| ||H_0||_F (closed form).  With
+    mean(t) = 127/7 the order of M is 6, 0, 1, 2, 5, 3, 4: every score row
+    must follow it, and the top 3 are blocks {0, 1, 6}."""
+    rng = np.random.default_rng(44)
+    nb, B, d = 7, 16, 6
+    L = nb * B
+    blk = np.arange(L) // B
+    base = rng.standard_normal((B, d))
+    base -= base.mean(axis=0)
+    centroid = rng.standard_normal(d)
+    vb = rng.standard_normal((B, d))
+    v = np.tile(vb, (nb, 1))
+    t = 2.0 ** np.arange(nb)
+    k = centroid[None, :] + base[np.arange(L) % B] * t[blk][:, None]
+    q = rng.standard_normal((L, d)) + 0.5
+    r = oracle.pisa_head(q, k, v, B, 3)
+    np.testing.assert_allclose(r["kbar"], np.tile(centroid, (nb, 1)), atol=1e-12)
+    want_M = np.abs(t - t.mean()) * np.linalg.norm(base.T @ vb)
+    np.testing.assert_allclose(r["M"], want_M, rtol=1e-10)
+    order = np.argsort(-want_M)
+    assert order.tolist() == [6, 0, 1, 2, 5, 3, 4]
+    for i in range(nb):
+        assert np.all(np.diff(r["scores"][i, order]) < 0), i
+    np.testing.assert_array_equal(r["sel"], np.tile([0, 1, 6], (nb, 1)))
+
+
 def test_keep_count_on_the_workloads():
     assert oracle.keep_count(1024, 64, 4 / 16) == 4
     assert oracle.keep_count(4608, 64, 0.25) == 18
