@@ -60,6 +60,35 @@ def effective_flops(cfg, sel):
     return exact, approx_per * sel.shape[0]
 
 
+def executed_mma_flops(cfg, sel):
+    """FLOPs of the MMAs the tensor-core fused kernel issues for selections
+    ``sel`` (bf16 path).  Every 128-row query tile runs one step per 128 keys
+    of its work list (one 128-token block, or two 64-token entries stacked),
+    then one step per 128 block centroids (nb rounded up to 128, padding and
+    selected columns masked but computed), each step an S = Q K^T and an
+    O += P V MMA group (2 x 2 x 128 x 128 x d), then q Hbar as a hi + lo pair
+    (2 x 2 x 128 x d x d).  The exact work list of a tile is the union of the
+    selections of its 128 / block query blocks."""
+    d, B, L, nb = cfg.d, cfg.block, cfg.L, cfg.nb
+    G = 128 // B
+    sel = sel.reshape(-1, nb, sel.shape[-1])
+    bh = sel.shape[0]
+    n_tiles = -(-L // 128)
+    ncent = -(-nb // 128)
+    if G == 1:
+        steps = np.full((bh, n_tiles), sel.shape[-1], dtype=np.int64)
+    else:
+        mask = np.zeros((bh, nb, nb), dtype=bool)
+        np.put_along_axis(mask, sel.astype(np.int64), True, axis=2)
+        pad = n_tiles * G - nb
+        if pad:
+            mask = np.concatenate([mask, np.zeros((bh, pad, nb), dtype=bool)], axis=1)
+        union = mask.reshape(bh, n_tiles, G, nb).any(axis=2)
+        steps = -(-union.sum(axis=2) // G)
+    per_step = 4.0 * 128 * 128 * d
+    return float(((steps + ncent) * per_step).sum() + bh * n_tiles * 4.0 * 128 * d * d)
+
+
 def stage_bytes(cfg, kk):
     """Algorithmic HBM bytes per launch of the streaming kernels."""
     bh, L, d, nb = cfg.batch * cfg.heads, cfg.L, cfg.d, cfg.nb
@@ -362,6 +391,27 @@ def whole_job_throughput(flops_per_rank: float, world: int, ms: float) -> float:
     return world * flops_per_rank / (ms * 1e-3) / 1e12
 
 
+def shard_range(n: int, world: int, rank: int):
+    """The contiguous (batch, head) slices [lo, hi) that ``rank`` of ``world``
+    computes when one batch is split by heads: every slice on exactly one
+    rank, shard sizes differing by at most one.  Each slice is an independent
+    problem (its statistics, routing and output rows use no other slice), so
+    the ranks exchange no data."""
+    if not 0 <= rank < world or n < world:
+        raise ValueError(f"cannot split {n} slices over {world} ranks")
+    return n * rank // world, n * (rank + 1) // world
+
+
+def sum_over_ranks(x: float, dist, device) -> float:
+    """Sum of ``x`` over all ranks (``x`` itself when not distributed)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
 def _source_sha(paths):
     import hashlib
     h = hashlib.sha256()
@@ -372,22 +422,30 @@ def _source_sha(paths):
 
 
 def stored_traffic(kernel, workload):
-    """DRAM bytes per launch from a committed ncu capture, or None when the
-    kernel's sources changed since the capture (or none was taken)."""
+    """(DRAM bytes per launch, how they were obtained) from a committed ncu
+    capture, or (None, reason) when the kernel's sources changed since the
+    capture (or none was taken)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
-        return None
+        return None, "no capture"
     with open(path) as f:
         table = json.load(f)
     e = table.get(kernel, {}).get(workload)
     if not e:
-        return None
+        return None, "no capture for this workload"
     try:
         if _source_sha(e["sources"]) != e["source_sha"]:
-            return None
+            return None, "kernel sources changed since the capture"
     except OSError:
-        return None
-    return e["bytes_per_launch"]
+        return None, "kernel sources missing"
+    return e["bytes_per_launch"], e.get("how", "")
+
+
+def spread(xs):
+    """Median, 10th and 90th percentile of a list of times."""
+    a = np.asarray(xs, dtype=np.float64)
+    return {"ms": float(np.median(a)), "p10_ms": float(np.percentile(a, 10)),
+            "p90_ms": float(np.percentile(a, 90)), "mean_ms": float(a.mean())}
 
 
 def main():
@@ -414,6 +472,9 @@ def main():
                     help="(batch, head) slices per chunk of the host-buffer pipeline")
     ap.add_argument("--heads", type=int, default=None,
                     help="run only the first N heads of the workload (profiling captures)")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="with N ranks: every rank runs the whole workload (replicas, weak scaling), "
+                         "or the batch x heads slices are split over the ranks (heads, strong scaling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -437,7 +498,15 @@ def main():
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
 
     # inputs first (the generator's worker pool is spawned, before any CUDA use)
-    q, k, v = generate(cfg)
+    full_cfg = cfg
+    sharded = args.shard == "heads" and world > 1
+    if sharded:
+        import dataclasses
+        lo, hi = shard_range(cfg.batch * cfg.heads, world, rank)
+        q, k, v = generate(cfg, heads=range(lo, hi))  # stored redraws, keyed by flat slice index
+        cfg = dataclasses.replace(cfg, batch=1, heads=hi - lo)
+    else:
+        q, k, v = generate(cfg)
 
     import torch
     import sparse_attention_diffusion_block_b200 as pisa
@@ -526,10 +595,13 @@ def main():
         dist.barrier()
     total_ms = t0.elapsed_time(t1)
     names = ["stats", "cov_norm", "select", "fused"]
-    stage_ms = {n: sum(e[i].elapsed_time(e[i + 1]) for e in evs) / K for i, n in enumerate(names)}
+    stage_times = {n: [e[i].elapsed_time(e[i + 1]) for e in evs] for i, n in enumerate(names)}
+    stage_ms = {n: sum(t) / K for n, t in stage_times.items()}
     total_ms = max_over_ranks(total_ms, dist, dev)
     ms = total_ms / K
-    value = whole_job_throughput(flops, world, ms)
+    # replicas: every rank moves the same FLOPs; heads: the ranks' shares add up
+    job_flops = sum_over_ranks(flops, dist, dev) if sharded else world * flops
+    value = job_flops / (ms * 1e-3) / 1e12
 
     # end to end through the public API with host buffers: pisa_attn_fwd_host
     # copies chunks of heads in, computes and copies out, overlapping the three
@@ -555,7 +627,7 @@ def main():
         torch.cuda.synchronize()
         e_ms = max_over_ranks(a.elapsed_time(z), dist, dev) / K
         in_bytes = sum(x.numel() * x.element_size() for x in (qd, kd, vd))
-        e2e = {"value": whole_job_throughput(flops, world, e_ms), "unit": "TFLOP/s", "ms_per_step": e_ms,
+        e2e = {"value": job_flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e_ms,
                "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out.numel() * out.element_size(),
                "api": f"pisa_attn_fwd_host, pinned host buffers, chunks of {args.e2e_chunk} heads"}
         del ws_host
@@ -563,21 +635,34 @@ def main():
     peaks = measured_peaks()
     fused_ms = stage_ms["fused"]
     achieved = flops / (fused_ms * 1e-3) / 1e12
-    peak = peaks["bf16_sustained"]
-    traffic = stored_traffic("fused", f"{cfg.name}:{cfg.heads}")
+    # the burst peak for a timed region under two seconds (the clocks have no
+    # time to settle at the power cap), the sustained one beyond
+    sustained = total_ms >= 2000.0
+    peak = peaks["bf16_sustained"] if sustained else peaks["bf16"]
+    traffic, traffic_how = stored_traffic("fused", f"{cfg.name}:{cfg.heads}")
+    executed = executed_mma_flops(cfg, sel_np) if cfg.dtype == "bf16" else None
     roofline = {"kernel": "fused attention (attn_fwd_with_sel)", "bound": "tensor",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "traffic": traffic,
-                "peak_source": f"{peaks['source']} sustained cuBLAS bf16 (timed inside a long step)"}
+                "traffic": traffic, "traffic_source": traffic_how,
+                "algorithmic_flops_per_launch": flops,
+                "peak_source": (f"{peaks['source']} {'sustained' if sustained else 'burst'} cuBLAS bf16: "
+                                f"timed region {total_ms / 1e3:.2f} s "
+                                f"({'>=' if sustained else '<'} 2 s)")}
+    if executed is not None:
+        ex_tf = executed / (fused_ms * 1e-3) / 1e12
+        roofline.update({"executed_mma_flops_per_launch": executed, "executed_TFLOP/s": ex_tf,
+                         "executed_frac": ex_tf / peak})
     sbytes = stage_bytes(cfg, kk)
     stages = {}
     for n in names:
-        ent = {"ms": stage_ms[n]}
+        ent = spread(stage_times[n])
         if n in sbytes:
-            gbs = sbytes[n] / (stage_ms[n] * 1e-3) / 1e9
+            gbs = sbytes[n] / (ent["ms"] * 1e-3) / 1e9
             ent.update({"algorithmic_bytes": sbytes[n], "GB/s": gbs, "frac_hbm": gbs / peaks["hbm"]})
         stages[n] = ent
-    stages["fused"]["TFLOP/s"] = achieved
+    stages["fused"]["TFLOP/s"] = flops / (stages["fused"]["ms"] * 1e-3) / 1e12
+    step_ms = [sum(e[i].elapsed_time(e[i + 1]) for i in range(4)) for e in evs]
+    stages["step"] = spread(step_ms)
 
     dense = None
     if rank == 0 and world == 1 and not args.no_dense_reference:
@@ -593,10 +678,15 @@ def main():
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "strong" if sharded else "weak",
             "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
-            "config": {"workload": describe(cfg, kk), "global_batch": world * cfg.batch,
-                       "seq_len": cfg.L, "parallelism": f"replicas x{world} (one full forward per GPU)",
+            "config": {"workload": describe(full_cfg, kk),
+                       "global_batch": full_cfg.batch if sharded else world * cfg.batch,
+                       "seq_len": cfg.L,
+                       "parallelism": (f"batch x heads split over {world} GPUs ({cfg.heads} slices on "
+                                       f"rank 0, no data-path collective)" if sharded else
+                                       f"replicas x{world} (one full forward per GPU)"),
                        "l2": f"inputs {3 * qd.numel() * qd.element_size() / 1e9:.2f} GB > L2 126 MB",
                        "route": args.route,
                        "launch_tuning": tuning or "built-in heuristics",

@@ -232,9 +232,12 @@ pisa_status pisa_attn_fwd_host(const void* q_host, const void* k_host, const voi
  * instead in one device array of PISA_NOALLOC_SCRATCH_BYTES compiled into the
  * library; every GPU that loads the library holds that memory until the
  * process exits.
- *   - A call whose scratch need, pisa_fused_workspace_size(batch, heads, L, d,
- *     block), exceeds PISA_NOALLOC_SCRATCH_BYTES is rejected with
- *     PISA_ERR_WORKSPACE before anything is launched.
+ *   - A bf16 call whose scratch need, pisa_fused_workspace_size(batch, heads,
+ *     L, d, block), exceeds PISA_NOALLOC_SCRATCH_BYTES is rejected with
+ *     PISA_ERR_WORKSPACE before anything is launched.  fp32 calls (the
+ *     CUDA-core kernel) use no scratch and have no such limit.
+ *   - The kernels and their operands are those of pisa_attn_fwd_with_sel, so
+ *     the output is bit-identical to it.
  *   - It calls no allocating routine (no cudaMalloc, cudaFree or library
  *     allocator).
  *   - The first call on each device looks up the array's device address
@@ -287,6 +290,22 @@ pisa_status pisa_get_tuning(int batch, int heads, int L, int d, int block, pisa_
  * rejected whole (PISA_ERR_INVALID_ARG) and changes nothing. */
 pisa_status pisa_tuning_save(const char* path);
 pisa_status pisa_tuning_load(const char* path);
+
+/* Sets the limit of the bounded waits in the tensor-core kernels on the
+ * current device, in nanoseconds of the GPU's global timer; 0 restores the
+ * default of 2 s.  Every mbarrier wait between the warps of a CTA (operand
+ * tiles landed, MMAs done, softmax done, work list ready) gives up after this
+ * long: the CTA then records PISA_ERR_TIMEOUT in the device error word,
+ * lets the copies and MMAs it already issued complete (a separate fixed 2 s
+ * bound that this setting does not shorten), frees its tensor memory and
+ * exits, so the context stays usable.  The result of such a call is
+ * undefined; pisa_device_status reports the timeout.  A limit shorter than
+ * the time a healthy copy or MMA takes (microseconds) makes ordinary calls
+ * time out: it exists to exercise that path in tests and to tighten the bound
+ * on a stuck kernel.  Applies to kernels launched after it; blocking:
+ * synchronises `stream`.  Not part of the method (the pages have no
+ * counterpart).  Returns PISA_OK or PISA_ERR_CUDA. */
+pisa_status pisa_set_wait_limit(uint64_t limit_ns, void* stream);
 
 /* Reads (and, when reset != 0, clears) the device error word that bounded
  * waits and index checks set.  Synchronises `stream`.  Returns PISA_OK,

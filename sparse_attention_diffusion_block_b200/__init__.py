@@ -10,7 +10,7 @@ block_stats, cov_norm, cov_norm_spectral, block_first_order, select, select_rout
 attn_fwd_with_sel, attn_fwd,
 attn_fwd_host, attn_fwd_with_sel_noalloc, keep_count, workspace_size, stats_workspace_size,
 fused_workspace_size, host_workspace_size, autotune, set_tuning, clear_tuning, get_tuning,
-tuning_save, tuning_load, device_status, status_string.
+tuning_save, tuning_load, set_wait_limit, device_status, status_string.
 """
 
 from __future__ import annotations
@@ -51,6 +51,7 @@ EXPORTS = (
     "pisa_device_status", "pisa_attn_fwd_with_sel_noalloc", "pisa_host_workspace_size",
     "pisa_attn_fwd_host", "pisa_select_route", "pisa_cov_norm_spectral", "pisa_autotune",
     "pisa_set_tuning", "pisa_get_tuning", "pisa_tuning_save", "pisa_tuning_load",
+    "pisa_set_wait_limit",
 )
 
 _p = ctypes.c_void_p
@@ -96,6 +97,7 @@ _lib_set_tuning = _sig("pisa_set_tuning", _i, _i, _i, _i, _i, _i, _TP)
 _lib_get_tuning = _sig("pisa_get_tuning", _i, _i, _i, _i, _i, _i, _TP)
 _lib_tuning_save = _sig("pisa_tuning_save", _i, ctypes.c_char_p)
 _lib_tuning_load = _sig("pisa_tuning_load", _i, ctypes.c_char_p)
+_lib_set_wait_limit = _sig("pisa_set_wait_limit", _i, ctypes.c_uint64, _p)
 _lib_fwd_host = _sig("pisa_attn_fwd_host", _i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _i, _p, _z, _p)
 
 
@@ -363,3 +365,11 @@ def launches(entry: str, dtype: torch.dtype = torch.bfloat16) -> int:
 
 def device_status(stream=None, reset: bool = True) -> int:
     return int(_lib_device_status(_stream(stream), 1 if reset else 0))
+
+
+def set_wait_limit(limit_ns: int = 0, stream=None) -> None:
+    """Limit of the tensor-core kernels' bounded waits on the current device,
+    in ns (0 restores the 2 s default).  Blocking."""
+    if limit_ns < 0:
+        raise ValueError("limit_ns must be >= 0")
+    _check(_lib_set_wait_limit(int(limit_ns), _stream(stream)), "set_wait_limit")

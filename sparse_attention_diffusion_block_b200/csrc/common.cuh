@@ -17,6 +17,11 @@ __device__ __forceinline__ void raise_device_error(int code) {
   atomicCAS(&g_error_word, 0, code);
 }
 
+// Limit of the bounded mbarrier waits, in ns of the global timer (one per
+// device; set by pisa_set_wait_limit, 2 s unless changed).
+constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;
+__device__ unsigned long long g_wait_limit_ns = kDefaultWaitLimitNs;
+
 __device__ __forceinline__ float to_float(float x) { return x; }
 __device__ __forceinline__ float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
 

@@ -385,10 +385,16 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     }
-    if (!ok && lane == 0) {
-      // let the copies already issued land before the CTA can exit
+    if (lane == 0) {
+      // the copies already issued land before the CTA can exit: the last load
+      // of each ring slot (the latest phase of its full barrier) and the last
+      // Q load of each tile buffer.  On the normal path the consumers have
+      // seen them, or will; after another role gave up nothing else waits
+      // for them.
       const int first = it > NS ? it - NS : 0;
-      for (int u = first; u < it; ++u) mbar_wait(&full[u % NS], (u / NS) & 1, abort);
+      for (int u = first; u < it; ++u) mbar_drain(&full[u % NS], (u / NS) & 1);
+      for (int x = 0; x < 2; ++x)
+        if (qloads[x] > 0) mbar_drain(&q_full[x], (qloads[x] - 1) & 1);
     }
    } else if (warp == 9) {
     // ================================================================ MMA issuer
@@ -505,9 +511,9 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         mma_commit_warp(&empty[h1]);
         if (lane == 0) mbar_arrive(&list_empty[slot]);
       }
+      // every MMA issued (on the normal path too) completes before TMEM is freed
       mma_commit_warp(mma_idle);
-      volatile int never = 0;
-      mbar_wait(mma_idle, 0, &never);
+      mbar_drain(mma_idle, 0);
     }
     __syncwarp();
    }

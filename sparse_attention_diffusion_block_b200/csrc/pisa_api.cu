@@ -9,6 +9,8 @@
 #include <tuple>
 #include <type_traits>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 #include "fused_simt.cuh"
 #include "fused_sm100.cuh"
@@ -30,6 +32,16 @@ struct Shape {
 };
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// NVTX range around the launches of one stage (host-side enqueue; a profiler
+// such as Nsight Systems lines it up with the kernels).  Without an attached
+// tool the push and pop are no-op calls.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // ------------------------------------------------------------------ launch tuning
 //
@@ -177,6 +189,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, u
 template <typename T, int D>
 pisa_status run_stats(const T* q, const T* k, const T* v, const Shape& s, float* qbar, float* kbar,
                       float* vsum, float* hbar, float* partial, cudaStream_t st) {
+  NvtxRange range("pisa.block_stats");
   const int J = stats_chunk(s), nc = stats_chunks(s);
   if constexpr (std::is_same<T, __nv_bfloat16>::value && D == 128) {
     CUtensorMap mQ, mK, mV;
@@ -219,6 +232,7 @@ int cov_chunk(const Shape& s) {
 template <typename T, int D, bool WRITE_H>
 pisa_status run_block_h(const T* k, const T* v, const Shape& s, const float* kbar, const float* vsum,
                         const float* hbar, float* out, cudaStream_t st) {
+  NvtxRange range(WRITE_H ? "pisa.block_first_order" : "pisa.cov_norm");
   if constexpr (std::is_same<T, __nv_bfloat16>::value && D == 128 && !WRITE_H) {
     CUtensorMap mK, mV;
     const uint32_t box = (uint32_t)s.block;
@@ -262,6 +276,7 @@ int select_rows(const Shape& s) {
 template <int D>
 pisa_status run_select(const float* qbar, const float* kbar, const float* M, const Shape& s, int k,
                        int32_t* sel, cudaStream_t st) {
+  NvtxRange range("pisa.select");
   const int nb = s.nb();
   const int R = select_rows(s);
   if (R < 1) return PISA_ERR_UNSUPPORTED;
@@ -277,6 +292,7 @@ template <typename T, int D>
 pisa_status run_fused(const T* q, const T* k, const T* v, T* out, const Shape& s, const float* kbar,
                       const float* vsum, const float* hbar, const int32_t* sel, int kk,
                       cudaStream_t st) {
+  NvtxRange range("pisa.fused");
   constexpr int TPR = 4, CH = 16, DS = D / TPR, RS = TPR * (DS + 4);
   const int nb = s.nb();
   const size_t smem = (2 * (size_t)CH * RS + (size_t)D * D + CH + (nb + 31) / 32) * sizeof(float);
@@ -321,6 +337,7 @@ template <int D, int KB>
 pisa_status run_fused_sm100(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                             __nv_bfloat16* out, const Shape& s, const float* kbar, const float* vsum,
                             const float* hbar, const int32_t* sel, int kk, void* ws, cudaStream_t st) {
+  NvtxRange range("pisa.fused");
   const int nb = s.nb(), nbp = padded_blocks(s), BH = s.BH();
   char* w = static_cast<char*>(ws);
   const size_t keys = align_up((size_t)BH * nbp * D * 2);
@@ -766,7 +783,8 @@ pisa_status pisa_attn_fwd_with_sel_noalloc(const void* q, const void* k, const v
   if (!valid_dtype(dtype)) return PISA_ERR_INVALID_ARG;
   if (k_sel < 1 || k_sel > s.nb()) return PISA_ERR_INVALID_ARG;
   if (!all_ok(q, k, v, out, kbar, vsum, hbar) || sel == nullptr) return PISA_ERR_INVALID_ARG;
-  if (fused_ws(s) > PISA_NOALLOC_SCRATCH_BYTES) return PISA_ERR_WORKSPACE;
+  // only the tensor-core (bf16) path takes scratch; the fp32 path uses none
+  if (dtype == PISA_BF16 && fused_ws(s) > PISA_NOALLOC_SCRATCH_BYTES) return PISA_ERR_WORKSPACE;
   void* scratch = nullptr;
   if (pisa_status e = noalloc_scratch(&scratch)) return e;
   return dispatch<FusedOp>(dtype, d, q, k, v, out, s, kbar, vsum, hbar, sel, k_sel, scratch,
@@ -940,6 +958,15 @@ pisa_status pisa_tuning_load(const char* path) {
   if (status != PISA_OK) return status;  // a malformed file changes nothing
   std::lock_guard<std::mutex> lock(g_tune_mutex);
   for (const auto& kv : got) g_tune[kv.first] = kv.second;
+  return PISA_OK;
+}
+
+pisa_status pisa_set_wait_limit(uint64_t limit_ns, void* stream) {
+  const unsigned long long v = limit_ns == 0 ? kDefaultWaitLimitNs : (unsigned long long)limit_ns;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaMemcpyToSymbolAsync(g_wait_limit_ns, &v, sizeof v, 0, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return PISA_ERR_CUDA;
   return PISA_OK;
 }
 

@@ -53,19 +53,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete.  Gives up after
-// kWaitLimitNs (or at once when *abort is set by another warp) and returns
-// false; the first timeout records PISA_ERR_TIMEOUT.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
-
+// Waits for the phase with the given parity to complete.  Gives up after the
+// device's wait limit (g_wait_limit_ns, read once per wait that has to spin),
+// or at once when *abort is set by another warp of the CTA, and returns false;
+// a wait that runs out sets *abort and records PISA_ERR_TIMEOUT.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t limit = *reinterpret_cast<volatile unsigned long long*>(&g_wait_limit_ns);
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit) {
       *abort = 1;
+      raise_device_error(PISA_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// Unwind-path wait for work this thread already issued (TMA copies into the
+// CTA's shared memory, its own MMAs): ignores the abort flag, so the copies
+// really land before the CTA can exit, and keeps a fixed 2 s bound of its own
+// that a short wait limit cannot cut.  Issued copies and MMAs complete in
+// microseconds; the bound only keeps a broken phase from hanging the CTA.
+constexpr uint64_t kDrainLimitNs = 2000000000ull;
+
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (global_timer_ns() - t0 > kDrainLimitNs) {
       raise_device_error(PISA_ERR_TIMEOUT);
       return false;
     }
@@ -188,6 +207,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
         "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
         "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
         "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+// 16 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15])
       : "r"(taddr));
 }
 

@@ -123,9 +123,11 @@ stats_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const int row = (j0 + jj) * KB;
         ok = load(&tmQ, row) && load(&tmK, row) && load(&tmV, row);
       }
-      if (!ok) {
+      {
+        // the last load of each ring slot lands before the CTA can exit (after
+        // another role gave up nothing else waits for it)
         const int first = it > NS ? it - NS : 0;
-        for (int u = first; u < it; ++u) mbar_wait(&full[u % NS], (u / NS) & 1, abort);
+        for (int u = first; u < it; ++u) mbar_drain(&full[u % NS], (u / NS) & 1);
       }
     }
   } else if (warp == 5) {
@@ -172,8 +174,7 @@ stats_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       }
       if (ok) mma_commit(h_final);
       mma_commit(mma_idle);
-      volatile int never = 0;
-      mbar_wait(mma_idle, 0, &never);
+      mbar_drain(mma_idle, 0);
     }
     __syncwarp();
   } else {
@@ -323,9 +324,11 @@ cov_norm_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         const int row = (j0 + jj) * KB;
         ok = load(&tmK, row) && load(&tmV, row);
       }
-      if (!ok) {
+      {
+        // the last load of each ring slot lands before the CTA can exit (after
+        // another role gave up nothing else waits for it)
         const int first = it > NS ? it - NS : 0;
-        for (int u = first; u < it; ++u) mbar_wait(&full[u % NS], (u / NS) & 1, abort);
+        for (int u = first; u < it; ++u) mbar_drain(&full[u % NS], (u / NS) & 1);
       }
     }
   } else if (warp == 5) {
@@ -358,8 +361,7 @@ cov_norm_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         mma_commit(&d_full[buf]);
       }
       mma_commit(mma_idle);
-      volatile int never = 0;
-      mbar_wait(mma_idle, 0, &never);
+      mbar_drain(mma_idle, 0);
     }
     __syncwarp();
   } else {

@@ -36,6 +36,19 @@ def oracle_head(q, k, v, B, kk, rows=None):
                             rows=rows)
 
 
+def oracle_routing(q, k, v, B, kk):
+    """The oracle's statistics and routing for one (batch, head), without the
+    output rows: returns dict(sel, Hbar, M)."""
+    q, k, v = (x.astype(np.float64) for x in (q, k, v))
+    s = 1.0 / math.sqrt(q.shape[1])
+    qbar, kbar, vsum, n = oracle.block_stats(q, k, v, B)
+    H = oracle.first_order_blocks(k, v, B, kbar)
+    Hbar = oracle.hbar_mean(H)
+    M = oracle.cov_norm(H, Hbar)
+    sel = oracle.select_topk(oracle.route_scores(qbar, kbar, M, n, s), kk)
+    return dict(sel=sel, Hbar=Hbar, M=M, H_scale=float(np.sqrt((H ** 2).sum(axis=(1, 2))).max()))
+
+
 def output_errors(gpu: np.ndarray, ref: np.ndarray):
     diff = gpu.astype(np.float64) - ref
     return float(np.abs(diff).max()), float(np.linalg.norm(diff) / np.linalg.norm(ref))
