@@ -374,6 +374,74 @@ def run_sweep(args):
     return 0
 
 
+ABLATION_SHAPES = ((4096, (4, 32, 32)), (8192, (8, 32, 32)))
+ABLATION_KEEP = (0.1, 0.25)
+
+
+def run_ablation(args):
+    """Accuracy / cost of the first-order term (the hybrid s beta_t (q_t Hbar)
+    against each unselected block's own s alpha_{t,j} (q_t H_j)) on small
+    video-like shapes: 8 heads, d=128, block 128, the 3-D generator on a
+    frames x 32 x 32 grid.  Both run on the same selections; the error is
+    measured against exact softmax attention (this library's fused kernel with
+    every block selected, which the oracle pins to dense attention), as
+    rel-L2 and max-abs over the whole output, and the time is that of the
+    attention call alone.  One JSON line."""
+    import torch
+    from workloads import Config
+    import sparse_attention_diffusion_block_b200 as pisa
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+
+    def timed(fn, reps=5):
+        fn()
+        torch.cuda.synchronize()
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            fn()
+        z.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(z) / reps
+
+    def errors(x, ref):
+        diff = (x.float() - ref.float())
+        return {"rel_l2": float(diff.norm() / ref.float().norm()), "max_abs": float(diff.abs().max())}
+
+    rows = []
+    for L, grid in ABLATION_SHAPES:
+        cfg = Config(f"ablation{L}", "bf16", 1, 8, L, 128, 128, seed=6, keep_ratio=0.1, kind="grid",
+                     grid=grid, R=16, A=1.5)
+        q, k, v = generate(cfg, redraws={})
+        qd, kd, vd = (torch.from_numpy(x).to(dev).to(torch.bfloat16) for x in (q, k, v))
+        B, nb = cfg.block, cfg.nb
+        qbar, kbar, vsum, hbar = pisa.block_stats(qd, kd, vd, B)
+        H = pisa.block_first_order(kd, vd, B, kbar, vsum)
+        M = pisa.cov_norm(kd, vd, B, kbar, vsum, hbar)
+        sel_all = torch.arange(nb, dtype=torch.int32, device=dev).expand(1, cfg.heads, nb, nb).contiguous()
+        dense = pisa.attn_fwd_with_sel(qd, kd, vd, B, kbar, vsum, hbar, sel_all)
+        for keep in ABLATION_KEEP:
+            kk = pisa.keep_count(L, B, keep)
+            sel = pisa.select(qbar, kbar, M, L, B, kk)
+            hyb = pisa.attn_fwd_with_sel(qd, kd, vd, B, kbar, vsum, hbar, sel)
+            blk = pisa.attn_fwd_blockwise_with_sel(qd, kd, vd, B, kbar, vsum, H, sel)
+            t_h = timed(lambda: pisa.attn_fwd_with_sel(qd, kd, vd, B, kbar, vsum, hbar, sel, out=hyb))
+            t_b = timed(lambda: pisa.attn_fwd_blockwise_with_sel(qd, kd, vd, B, kbar, vsum, H, sel, out=blk),
+                        reps=2)
+            rows.append({"L": L, "keep": keep, "k": kk,
+                         "hybrid": {"ms": t_h, **errors(hyb, dense)},
+                         "blockwise": {"ms": t_b, **errors(blk, dense)}})
+        if pisa.device_status() != 0:
+            raise RuntimeError("device status set during the ablation")
+        del qd, kd, vd, H, dense, sel_all
+        torch.cuda.empty_cache()
+    print(json.dumps({"ablation": "first-order term: hybrid (Hbar, tensor cores) vs per-block H_j (CUDA cores); "
+                                  "error against exact softmax attention", "heads": 8, "d": 128, "block": 128,
+                      "rows": rows}), flush=True)
+    return 0
+
+
 def max_over_ranks(x: float, dist, device) -> float:
     """The maximum of ``x`` over all ranks (the slowest rank's time); ``x``
     itself when not distributed."""
@@ -466,6 +534,9 @@ def main():
                          "the pooled score, or the covariance score with the spectral norm")
     ap.add_argument("--sweep", action="store_true",
                     help="sequence-length x density sweep (4K-32K tokens) instead of the bench line")
+    ap.add_argument("--ablation", action="store_true",
+                    help="first-order term ablation (hybrid vs per-block H_j) on small shapes instead of the "
+                         "bench line")
     ap.add_argument("--no-dense-reference", action="store_true",
                     help="skip the dense-attention context (every block selected; torch SDPA)")
     ap.add_argument("--e2e-chunk", type=int, default=2,
@@ -487,6 +558,8 @@ def main():
 
     if args.sweep:
         return run_sweep(args)
+    if args.ablation:
+        return run_ablation(args)
     if args.impl == "reference":
         import oracle  # reference arm: the oracle as it stands
         return run_reference(args, cfg, oracle.keep_count(cfg.L, cfg.block, cfg.keep_ratio))

@@ -216,6 +216,24 @@ pisa_status pisa_attn_fwd_host(const void* q_host, const void* k_host, const voi
                                int d, int block, float keep_ratio, int chunk, void* workspace,
                                size_t workspace_bytes, void* stream);
 
+/* The forward with each unselected block's own first-order term instead of
+ * the shared one: N_t = sum_{S_i} e^{x} v + sum_{j in U_i} alpha_{t,j}
+ * (sigma_j + s q_t H_j), D_t as in pisa_attn_fwd_with_sel (gist.science
+ * technical summary, section 2: the hybrid-order paragraph starts from these
+ * per-block terms and replaces H_j by Hbar to avoid loading them).  For the
+ * accuracy / cost comparison between the two: it costs (nb - k) d^2
+ * multiply-adds per query row and reads H, so it runs on CUDA cores and is
+ * meant for small shapes (a few thousand tokens); the production path is
+ * pisa_attn_fwd_with_sel.
+ *   H:   [batch, heads, nb, d, d] float32, the block-wise first-order
+ *        matrices H_j (pisa_block_first_order).
+ *   Other arguments as pisa_attn_fwd_with_sel; no workspace.  Validation
+ *   errors as there. */
+pisa_status pisa_attn_fwd_blockwise_with_sel(const void* q, const void* k, const void* v, void* out,
+                                             pisa_dtype dtype, int batch, int heads, int L, int d,
+                                             int block, const float* kbar, const float* vsum,
+                                             const float* H, const int32_t* sel, int k_sel, void* stream);
+
 /* Size in bytes of the fixed device scratch array used by
  * pisa_attn_fwd_with_sel_noalloc (32 MiB). */
 #define PISA_NOALLOC_SCRATCH_BYTES (32ull * 1024ull * 1024ull)
@@ -264,7 +282,10 @@ pisa_status pisa_attn_fwd_with_sel_noalloc(const void* q, const void* k, const v
  * they would change results. */
 typedef struct pisa_tuning {
   int cov_blocks_per_cta;   /* >= 0 */
-  int select_rows_per_cta;  /* 0..32, capped by shared memory */
+  int select_rows_per_cta;  /* 0..32: the tensor-core routing kernel runs 32 (values
+                               above 16 or 0) or 16 (1..16) query blocks per CTA; the
+                               CUDA-core one, for nb too large for the former, up to
+                               what fits in shared memory */
   int fused_ctas;           /* >= 0, capped by the SM count and the pairs of query tiles */
 } pisa_tuning;
 

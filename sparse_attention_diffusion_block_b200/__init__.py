@@ -7,7 +7,7 @@ loudly when the library has not been built.
 
 Entry points mirror the C names (without the ``pisa_`` prefix):
 block_stats, cov_norm, cov_norm_spectral, block_first_order, select, select_route,
-attn_fwd_with_sel, attn_fwd,
+attn_fwd_with_sel, attn_fwd_blockwise_with_sel, attn_fwd,
 attn_fwd_host, attn_fwd_with_sel_noalloc, keep_count, workspace_size, stats_workspace_size,
 fused_workspace_size, host_workspace_size, autotune, set_tuning, clear_tuning, get_tuning,
 tuning_save, tuning_load, set_wait_limit, device_status, status_string.
@@ -51,7 +51,7 @@ EXPORTS = (
     "pisa_device_status", "pisa_attn_fwd_with_sel_noalloc", "pisa_host_workspace_size",
     "pisa_attn_fwd_host", "pisa_select_route", "pisa_cov_norm_spectral", "pisa_autotune",
     "pisa_set_tuning", "pisa_get_tuning", "pisa_tuning_save", "pisa_tuning_load",
-    "pisa_set_wait_limit",
+    "pisa_set_wait_limit", "pisa_attn_fwd_blockwise_with_sel",
 )
 
 _p = ctypes.c_void_p
@@ -97,6 +97,8 @@ _lib_set_tuning = _sig("pisa_set_tuning", _i, _i, _i, _i, _i, _i, _TP)
 _lib_get_tuning = _sig("pisa_get_tuning", _i, _i, _i, _i, _i, _i, _TP)
 _lib_tuning_save = _sig("pisa_tuning_save", _i, ctypes.c_char_p)
 _lib_tuning_load = _sig("pisa_tuning_load", _i, ctypes.c_char_p)
+_lib_fwd_blockwise = _sig("pisa_attn_fwd_blockwise_with_sel", _i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i,
+                          _p, _p, _p, _p, _i, _p)
 _lib_set_wait_limit = _sig("pisa_set_wait_limit", _i, ctypes.c_uint64, _p)
 _lib_fwd_host = _sig("pisa_attn_fwd_host", _i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _i, _p, _z, _p)
 
@@ -269,6 +271,20 @@ def attn_fwd_with_sel_noalloc(q, k, v, block, kbar, vsum, hbar, sel, out=None, s
     _check(_lib_fwd_sel_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), b, h, L, d, block,
                                 _ptr(kbar), _ptr(vsum), _ptr(hbar), _ptr(sel), int(sel.shape[-1]),
                                 _stream(stream)), "pisa_attn_fwd_with_sel_noalloc")
+    return out
+
+
+def attn_fwd_blockwise_with_sel(q, k, v, block, kbar, vsum, H, sel, out=None, stream=None):
+    """The forward with each unselected block's own first-order term s alpha
+    (q_t H_j) instead of s beta (q_t Hbar); H from block_first_order.  CUDA
+    cores, (nb - k) d^2 per row: a comparison variant for small shapes."""
+    _need_cuda(q, k, v, kbar, vsum, H, sel)
+    b, h, L, d = _qkv_shape(q)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(_lib_fwd_blockwise(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), b, h, L, d, block,
+                              _ptr(kbar), _ptr(vsum), _ptr(H), _ptr(sel), int(sel.shape[-1]),
+                              _stream(stream)), "pisa_attn_fwd_blockwise_with_sel")
     return out
 
 

@@ -13,15 +13,61 @@
 
 namespace pisa {
 
+// o[0..DS) += fo * (q_t H)[sl*DS .. sl*DS+DS) for the row whose TPR threads
+// hold q_t in slices: each thread forms the partial products of its own slice
+// of q_t with every column block, and the TPR partials of a column block are
+// summed with shuffles.  Hs: a D x D matrix in shared memory (row = key dim).
+template <int D, int TPR>
+__device__ __forceinline__ void add_q_times_h(const float* __restrict__ Hs, const float* qr, float* o, float fo,
+                                              int sl) {
+  constexpr int DS = D / TPR;
+#pragma unroll 1
+  for (int g = 0; g < TPR; ++g) {
+    float part[DS];
+#pragma unroll
+    for (int c = 0; c < DS; ++c) part[c] = 0.f;
+#pragma unroll 4
+    for (int a = 0; a < DS; ++a) {
+      const float qa = qr[a];
+      const float* hrow = Hs + (sl * DS + a) * D + g * DS;
+#pragma unroll
+      for (int c = 0; c < DS; c += 4) {
+        const float4 w = *reinterpret_cast<const float4*>(hrow + c);
+        part[c] = fmaf(qa, w.x, part[c]);
+        part[c + 1] = fmaf(qa, w.y, part[c + 1]);
+        part[c + 2] = fmaf(qa, w.z, part[c + 2]);
+        part[c + 3] = fmaf(qa, w.w, part[c + 3]);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < DS; ++c) {
+#pragma unroll
+      for (int off = 1; off < TPR; off <<= 1) part[c] += __shfl_xor_sync(0xffffffffu, part[c], off);
+    }
+    if (sl == g) {
+#pragma unroll
+      for (int c = 0; c < DS; ++c) o[c] = fmaf(fo, part[c], o[c]);
+    }
+  }
+}
+
 // One CTA per (query block i, bh); TPR threads per query row, each owning
 // DS = D / TPR consecutive dimensions of q_t and O_t.  Keys are staged in
 // shared memory CH at a time, fp32, laid out [CH][TPR][DS + 4].
-template <typename T, int D, int TPR, int CH>
+//
+// BLOCKWISE selects the first-order term before hybridisation (gist.science
+// summary, section 2, the hybrid-order paragraph starts from it): every
+// unselected block keeps its own H_j, N_t += s alpha_{t,j} (q_t H_j), instead
+// of the shared s beta_t (q_t Hbar).  `first` is then H [BH][nb][D][D]; the
+// term is folded into the same running numerator as the block's value sum.
+// It costs |U_i| D^2 multiply-adds per row: a comparison variant for small
+// shapes, not the production path.  Otherwise `first` is Hbar [BH][D][D].
+template <typename T, int D, int TPR, int CH, bool BLOCKWISE = false>
 __global__ void __launch_bounds__(512, 1)
 fused_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                   T* __restrict__ out, int L, int B, int nb, int kk,
                   const float* __restrict__ kbar, const float* __restrict__ vsum,
-                  const float* __restrict__ hbar, const int32_t* __restrict__ sel, float scale) {
+                  const float* __restrict__ first, const int32_t* __restrict__ sel, float scale) {
   constexpr int DS = D / TPR;
   constexpr int SS = DS + 4;            // padded slice stride
   constexpr int RS = TPR * SS;          // padded row stride
@@ -174,16 +220,19 @@ fused_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
       cmax = fmaxf(cmax, y[c]);
     }
     const float m_new = fmaxf(m, cmax);
-    if (m_new == -INFINITY) continue;  // nothing unselected in this tile yet
-    const float corr = exp2f(m - m_new);
+    // nothing unselected in this tile yet (uniform: the CTA's rows share S_i)
+    if (m_new == -INFINITY && !BLOCKWISE) continue;
+    const float corr = m_new == -INFINITY ? 1.f : exp2f(m - m_new);
     l *= corr;
     beta *= corr;
 #pragma unroll
     for (int e2 = 0; e2 < DS; ++e2) o[e2] *= corr;
     m = m_new;
+    float alpha[CH];
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
-      const float a = exp2f(y[c] - m);
+      const float a = m == -INFINITY ? 0.f : exp2f(y[c] - m);
+      alpha[c] = a;
       beta += a;
       l = fmaf(nj_s[c], a, l);
       const float* vr = Vt + c * RS + sl * SS;
@@ -196,41 +245,29 @@ fused_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
         o[e2 + 3] = fmaf(a, w.w, o[e2 + 3]);
       }
     }
-  }
-
-  // ---- phase 3: global first-order correction  O += s * beta * (q Hbar)
-  __syncthreads();
-  const float* hb = hbar + (size_t)bh * D * D;
-  for (int e = threadIdx.x; e < D * D; e += blockDim.x) Hs[e] = hb[e];
-  __syncthreads();
-  const float fo = scale * beta;
-#pragma unroll 1
-  for (int g = 0; g < TPR; ++g) {
-    float part[DS];
-#pragma unroll
-    for (int c = 0; c < DS; ++c) part[c] = 0.f;
-#pragma unroll 4
-    for (int a = 0; a < DS; ++a) {
-      const float qa = qr[a];
-      const float* hrow = Hs + (sl * DS + a) * D + g * DS;
-#pragma unroll
-      for (int c = 0; c < DS; c += 4) {
-        const float4 w = *reinterpret_cast<const float4*>(hrow + c);
-        part[c] = fmaf(qa, w.x, part[c]);
-        part[c + 1] = fmaf(qa, w.y, part[c + 1]);
-        part[c + 2] = fmaf(qa, w.z, part[c + 2]);
-        part[c + 3] = fmaf(qa, w.w, part[c + 3]);
+    if constexpr (BLOCKWISE) {
+      // each unselected block's own first-order term, weighted like its value
+      // sum: O += s alpha_{t,j} (q_t H_j)
+      for (int c = 0; c < cn; ++c) {
+        const int j = j0 + c;
+        if ((mask[j >> 5] >> (j & 31)) & 1u) continue;  // selected: exact above
+        __syncthreads();
+        const float* hj = first + ((size_t)bh * nb + j) * D * D;
+        for (int e = threadIdx.x; e < D * D / 4; e += blockDim.x)
+          reinterpret_cast<float4*>(Hs)[e] = reinterpret_cast<const float4*>(hj)[e];
+        __syncthreads();
+        add_q_times_h<D, TPR>(Hs, qr, o, scale * alpha[c], sl);
       }
     }
-#pragma unroll
-    for (int c = 0; c < DS; ++c) {
-#pragma unroll
-      for (int off = 1; off < TPR; off <<= 1) part[c] += __shfl_xor_sync(0xffffffffu, part[c], off);
-    }
-    if (sl == g) {
-#pragma unroll
-      for (int c = 0; c < DS; ++c) o[c] = fmaf(fo, part[c], o[c]);
-    }
+  }
+
+  if constexpr (!BLOCKWISE) {
+    // ---- phase 3: global first-order correction  O += s * beta * (q Hbar)
+    __syncthreads();
+    const float* hb = first + (size_t)bh * D * D;
+    for (int e = threadIdx.x; e < D * D; e += blockDim.x) Hs[e] = hb[e];
+    __syncthreads();
+    add_q_times_h<D, TPR>(Hs, qr, o, scale * beta, sl);
   }
 
   if (active) {

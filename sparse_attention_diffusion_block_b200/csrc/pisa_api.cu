@@ -16,6 +16,7 @@
 #include "fused_sm100.cuh"
 #include "route_variants.cuh"
 #include "select.cuh"
+#include "select_sm100.cuh"
 #include "stats_simt.cuh"
 #include "stats_sm100.cuh"
 
@@ -258,7 +259,32 @@ pisa_status run_block_h(const T* k, const T* v, const Shape& s, const float* kba
   return last_launch();
 }
 
-// Largest routing tile that fits: R rows of nb keys in 150 KB, at most 32.
+// Routing on the tensor cores: R = 32 query blocks per CTA (the MMA's N), or
+// 16 when the [R][nb] key buffer of 32 leaves no room for two 32 KB stages.
+// Returns (R, stages), or R = 0 when even R = 16 does not fit (then the
+// CUDA-core routing kernel, which needs no staging, takes the shape).
+constexpr size_t kSmemMax = 227 * 1024;
+
+template <int D, int R>
+int select_tc_stages(int nb) {
+  for (int ns = 4; ns >= 2; --ns)
+    if (SelectTcLayout<D, R>::bytes(ns, nb) <= kSmemMax) return ns;
+  return 0;
+}
+
+template <int D>
+void select_tc_plan(int nb, int tuned_r, int* R, int* ns) {
+  *R = 0;
+  *ns = 0;
+  const bool want16 = tuned_r > 0 && tuned_r <= 16;
+  if (!want16 && (*ns = select_tc_stages<D, 32>(nb)) > 0) {
+    *R = 32;
+  } else if ((*ns = select_tc_stages<D, 16>(nb)) > 0) {
+    *R = 16;
+  }
+}
+
+// Largest routing tile of the CUDA-core kernel: R rows of nb keys in 140 KB, at most 32.
 int select_rows_max(int nb) {
   // the key buffer (R x nb words) beside the fixed tiles, within 227 KB
   const long long budget = 140 * 1024;
@@ -273,11 +299,32 @@ int select_rows(const Shape& s) {
   return (tuned > 0 && tuned < cap) ? tuned : cap;
 }
 
+bool make_map_f32(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer,
+                  uint32_t box_rows);
+
+template <int D, int R>
+pisa_status launch_select_tc(const float* qbar, const float* kbar, const float* M, const Shape& s, int k,
+                             int ns, int32_t* sel, cudaStream_t st) {
+  const int nb = s.nb();
+  CUtensorMap mK;
+  if (!make_map_f32(&mK, kbar, D, nb, s.BH(), 128)) return PISA_ERR_CUDA;
+  const size_t smem = SelectTcLayout<D, R>::bytes(ns, nb);
+  if (!set_smem(select_sm100_kernel<D, R>, smem)) return PISA_ERR_CUDA;
+  const float scale = 1.0f / sqrtf((float)D);
+  select_sm100_kernel<D, R><<<dim3((nb + R - 1) / R, s.BH()), kSelTcThreads, smem, st>>>(
+      mK, qbar, M, s.L, s.block, nb, k, ns, scale, sel);
+  return last_launch();
+}
+
 template <int D>
 pisa_status run_select(const float* qbar, const float* kbar, const float* M, const Shape& s, int k,
                        int32_t* sel, cudaStream_t st) {
   NvtxRange range("pisa.select");
   const int nb = s.nb();
+  int Rtc = 0, ns = 0;
+  select_tc_plan<D>(nb, tuning_for(s.BH(), s.L, s.d, s.block).select_r, &Rtc, &ns);
+  if (Rtc == 32) return launch_select_tc<D, 32>(qbar, kbar, M, s, k, ns, sel, st);
+  if (Rtc == 16) return launch_select_tc<D, 16>(qbar, kbar, M, s, k, ns, sel, st);
   const int R = select_rows(s);
   if (R < 1) return PISA_ERR_UNSUPPORTED;
   const size_t smem = select_smem_bytes(D, R, nb);
@@ -302,6 +349,32 @@ pisa_status run_fused(const T* q, const T* k, const T* v, T* out, const Shape& s
       q, k, v, out, s.L, s.block, nb, kk, kbar, vsum, hbar, sel, scale);
   return last_launch();
 }
+
+// The CUDA-core fused kernel with each unselected block's own first-order
+// term (H: [BH][nb][D][D]), either dtype.
+template <typename T, int D>
+pisa_status run_fused_blockwise(const T* q, const T* k, const T* v, T* out, const Shape& s, const float* kbar,
+                                const float* vsum, const float* H, const int32_t* sel, int kk, cudaStream_t st) {
+  NvtxRange range("pisa.fused_blockwise");
+  constexpr int TPR = 4, CH = 16, DS = D / TPR, RS = TPR * (DS + 4);
+  const int nb = s.nb();
+  const size_t smem = (2 * (size_t)CH * RS + (size_t)D * D + CH + (nb + 31) / 32) * sizeof(float);
+  if (!set_smem(fused_simt_kernel<T, D, TPR, CH, true>, smem)) return PISA_ERR_CUDA;
+  const float scale = 1.0f / sqrtf((float)D);
+  fused_simt_kernel<T, D, TPR, CH, true><<<dim3(nb, s.BH()), s.block * TPR, smem, st>>>(
+      q, k, v, out, s.L, s.block, nb, kk, kbar, vsum, H, sel, scale);
+  return last_launch();
+}
+
+template <typename T, int D>
+struct FusedBlockwiseOp {
+  static pisa_status run(const void* q, const void* k, const void* v, void* out, const Shape& s,
+                         const float* kbar, const float* vsum, const float* H, const int32_t* sel, int kk,
+                         cudaStream_t st) {
+    return run_fused_blockwise<T, D>((const T*)q, (const T*)k, (const T*)v, (T*)out, s, kbar, vsum, H, sel, kk,
+                                     st);
+  }
+};
 
 using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -329,6 +402,21 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, u
   const cuuint32_t box[3] = {64, box_rows, 1};
   const cuuint32_t es[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D fp32 map over [outer][rows][inner] with 32-element (128-byte) swizzled
+// boxes of `box_rows` rows; reads outside [0, rows) return zeros.
+bool make_map_f32(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer,
+                  uint32_t box_rows) {
+  EncodeTiled fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {inner, rows, outer};
+  const cuuint64_t strides[2] = {inner * 4, inner * rows * 4};
+  const cuuint32_t box[3] = {32, box_rows, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -774,6 +862,18 @@ pisa_status pisa_attn_fwd_with_sel(const void* q, const void* k, const void* v, 
                            (cudaStream_t)stream);
 }
 
+pisa_status pisa_attn_fwd_blockwise_with_sel(const void* q, const void* k, const void* v, void* out,
+                                             pisa_dtype dtype, int batch, int heads, int L, int d, int block,
+                                             const float* kbar, const float* vsum, const float* H,
+                                             const int32_t* sel, int k_sel, void* stream) {
+  const Shape s{batch, heads, L, d, block};
+  if (pisa_status e = check_shape(s)) return e;
+  if (!valid_dtype(dtype)) return PISA_ERR_INVALID_ARG;
+  if (k_sel < 1 || k_sel > s.nb()) return PISA_ERR_INVALID_ARG;
+  if (!all_ok(q, k, v, out, kbar, vsum, H) || sel == nullptr) return PISA_ERR_INVALID_ARG;
+  return dispatch<FusedBlockwiseOp>(dtype, d, q, k, v, out, s, kbar, vsum, H, sel, k_sel, (cudaStream_t)stream);
+}
+
 pisa_status pisa_attn_fwd_with_sel_noalloc(const void* q, const void* k, const void* v, void* out,
                                            pisa_dtype dtype, int batch, int heads, int L, int d, int block,
                                            const float* kbar, const float* vsum, const float* hbar,
@@ -868,10 +968,18 @@ pisa_status pisa_autotune(const void* q, const void* k, const void* v, void* out
                                (const float*)c.hbar, c.M, st);
   });
   if (e) return e;
-  // routing: rows per CTA, up to what fits in shared memory
+  // routing: rows per CTA; the tensor-core kernel runs 32 or 16 (the MMA's N),
+  // the CUDA-core one up to what fits in shared memory
+  int rtc = 0, ns = 0;
+  if (d == 128) select_tc_plan<128>(nb, 0, &rtc, &ns); else select_tc_plan<64>(nb, 0, &rtc, &ns);
   const int rmax = select_rows_max(nb);
   int cr[4] = {rmax, rmax >= 24 ? 24 : rmax, rmax >= 16 ? 16 : rmax, rmax >= 8 ? 8 : rmax};
-  e = pick(key, &t, &Tuning::select_r, cr, 4, st, [&] {
+  const int ncr = rtc == 32 ? 2 : rtc == 16 ? 1 : 4;
+  if (rtc > 0) {
+    cr[0] = rtc;
+    cr[1] = 16;
+  }
+  e = pick(key, &t, &Tuning::select_r, cr, ncr, st, [&] {
     return d == 128 ? run_select<128>(c.qbar, c.kbar, c.M, s, kk, c.sel, st)
                     : run_select<64>(c.qbar, c.kbar, c.M, s, kk, c.sel, st);
   });

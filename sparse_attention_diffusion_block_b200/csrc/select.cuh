@@ -17,6 +17,104 @@ __device__ __forceinline__ uint32_t orderable_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// The k largest of the nb keys kr[0..nb) (exact ties to the smaller index),
+// written to out[0..k) in ascending index order.  One warp per row, every lane
+// calls it.  An MSB-first bitwise search finds the k-th largest key (a 0 key
+// stands for "no block" and is never counted, since every candidate is >= 1);
+// then the keys above it and the first ties below it are compacted in index
+// order.  NR keys per lane are held in registers (nb <= 32 NR).
+template <int NR>
+__device__ __forceinline__ uint32_t kth_largest_in_regs(const uint32_t* __restrict__ kr, int nb, int kk,
+                                                       int lane) {
+  uint32_t kv[NR];
+  uint32_t mx = 0u, mn = 0xffffffffu;
+#pragma unroll
+  for (int m = 0; m < NR; ++m) {
+    const int j = lane + 32 * m;
+    kv[m] = (j < nb) ? kr[j] : 0u;
+    if (j < nb) {
+      mx = max(mx, kv[m]);
+      mn = min(mn, kv[m]);
+    }
+  }
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  mn = __reduce_min_sync(0xffffffffu, mn);
+  // the k-th largest lies in [mn, mx], so it shares their common high bits
+  const uint32_t diff = mx ^ mn;
+  if (diff == 0u) return mx;
+  const int top = 31 - __clz(diff);
+  uint32_t prefix = (top == 31) ? 0u : (mx & ~((2u << top) - 1u));
+  for (int bit = top; bit >= 0; --bit) {
+    const uint32_t cand = prefix | (1u << bit);
+    int cnt = 0;
+#pragma unroll
+    for (int m = 0; m < NR; ++m) cnt += (kv[m] >= cand);
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
+    if (cnt >= kk) prefix = cand;
+  }
+  return prefix;
+}
+
+__device__ __forceinline__ void topk_row_ascending(const uint32_t* __restrict__ kr, int nb, int kk, int lane,
+                                                   int32_t* __restrict__ out) {
+  uint32_t thr;  // k-th largest key
+  if (nb <= 256) {
+    thr = kth_largest_in_regs<8>(kr, nb, kk, lane);
+  } else if (nb <= 512) {
+    thr = kth_largest_in_regs<16>(kr, nb, kk, lane);
+  } else if (nb <= 768) {
+    thr = kth_largest_in_regs<24>(kr, nb, kk, lane);
+  } else if (nb <= 1024) {
+    thr = kth_largest_in_regs<32>(kr, nb, kk, lane);
+  } else {
+    uint32_t prefix = 0;
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = prefix | (1u << bit);
+      int cnt = 0;
+      for (int j = lane; j < nb; j += 32) cnt += (kr[j] >= cand);
+      cnt = __reduce_add_sync(0xffffffffu, cnt);
+      if (cnt >= kk) prefix = cand;
+    }
+    thr = prefix;
+  }
+  const int C = (nb + 31) / 32;  // contiguous chunk of indices per lane
+  const int jb = min(nb, lane * C), je = min(nb, jb + C);
+  int n_gt = 0, n_eq = 0;
+  for (int j = jb; j < je; ++j) {
+    n_gt += (kr[j] > thr);
+    n_eq += (kr[j] == thr);
+  }
+  const int tot_gt = __reduce_add_sync(0xffffffffu, n_gt);
+  const int need = kk - tot_gt;  // ties taken, lowest indices first
+  // exclusive scans over lanes
+  int eq_before = n_eq, sel_before;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, eq_before, o);
+    if (lane >= o) eq_before += y;
+  }
+  eq_before -= n_eq;
+  const int take_eq = max(0, min(n_eq, need - eq_before));
+  const int mine = n_gt + take_eq;
+  sel_before = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, sel_before, o);
+    if (lane >= o) sel_before += y;
+  }
+  sel_before -= mine;
+  int pos = sel_before, eq_taken = 0;
+  for (int j = jb; j < je; ++j) {
+    const uint32_t key = kr[j];
+    bool take = key > thr;
+    if (key == thr && eq_taken < take_eq) {
+      take = true;
+      ++eq_taken;
+    }
+    if (take) out[pos++] = j;
+  }
+}
+
 constexpr int kSelectThreads = 512;  // 16 warps
 constexpr int kSelectKT = 128;       // key blocks per score tile
 
@@ -119,92 +217,9 @@ select_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
   }
   __syncthreads();
 
-  // Phase 2: per-row selection.
-  const int C = (nb + 31) / 32;  // contiguous chunk of indices per lane
-  for (int r = warp; r < rows; r += NW) {
-    const uint32_t* kr = keys + r * nb;
-    uint32_t thr;  // k-th largest key
-    if (nb <= 1024) {
-      // keys in registers (j = lane + 32 m; a 0 key stands for "no block" and
-      // is never counted since every candidate is >= 1)
-      uint32_t kv[32];
-      uint32_t mx = 0u, mn = 0xffffffffu;
-#pragma unroll
-      for (int m = 0; m < 32; ++m) {
-        const int j = lane + 32 * m;
-        kv[m] = (j < nb) ? kr[j] : 0u;
-        if (j < nb) {
-          mx = max(mx, kv[m]);
-          mn = min(mn, kv[m]);
-        }
-      }
-      mx = __reduce_max_sync(0xffffffffu, mx);
-      mn = __reduce_min_sync(0xffffffffu, mn);
-      // the k-th largest lies in [mn, mx], so it shares their common high bits
-      const uint32_t diff = mx ^ mn;
-      if (diff == 0u) {
-        thr = mx;
-      } else {
-        const int top = 31 - __clz(diff);
-        uint32_t prefix = (top == 31) ? 0u : (mx & ~((2u << top) - 1u));
-        for (int bit = top; bit >= 0; --bit) {
-          const uint32_t cand = prefix | (1u << bit);
-          int cnt = 0;
-#pragma unroll
-          for (int m = 0; m < 32; ++m) cnt += (kv[m] >= cand);
-          cnt = __reduce_add_sync(0xffffffffu, cnt);
-          if (cnt >= kk) prefix = cand;
-        }
-        thr = prefix;
-      }
-    } else {
-      uint32_t prefix = 0;
-      for (int bit = 31; bit >= 0; --bit) {
-        const uint32_t cand = prefix | (1u << bit);
-        int cnt = 0;
-        for (int j = lane; j < nb; j += 32) cnt += (kr[j] >= cand);
-        cnt = __reduce_add_sync(0xffffffffu, cnt);
-        if (cnt >= kk) prefix = cand;
-      }
-      thr = prefix;
-    }
-    const int jb = lane * C, je = min(nb, jb + C);
-    int n_gt = 0, n_eq = 0;
-    for (int j = jb; j < je; ++j) {
-      n_gt += (kr[j] > thr);
-      n_eq += (kr[j] == thr);
-    }
-    const int tot_gt = __reduce_add_sync(0xffffffffu, n_gt);
-    const int need = kk - tot_gt;  // ties taken, lowest indices first
-    // exclusive scans over lanes
-    int eq_before = n_eq, sel_before;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, eq_before, o);
-      if (lane >= o) eq_before += y;
-    }
-    eq_before -= n_eq;
-    const int take_eq = max(0, min(n_eq, need - eq_before));
-    const int mine = n_gt + take_eq;
-    sel_before = mine;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, sel_before, o);
-      if (lane >= o) sel_before += y;
-    }
-    sel_before -= mine;
-    int32_t* out = sel + ((size_t)bh * nb + i0 + r) * kk;
-    int pos = sel_before, eq_taken = 0;
-    for (int j = jb; j < je; ++j) {
-      const uint32_t key = kr[j];
-      bool take = key > thr;
-      if (key == thr && eq_taken < take_eq) {
-        take = true;
-        ++eq_taken;
-      }
-      if (take) out[pos++] = j;
-    }
-  }
+  // Phase 2: per-row selection, one warp per row.
+  for (int r = warp; r < rows; r += NW)
+    topk_row_ascending(keys + r * nb, nb, kk, lane, sel + ((size_t)bh * nb + i0 + r) * kk);
 }
 
 }  // namespace pisa

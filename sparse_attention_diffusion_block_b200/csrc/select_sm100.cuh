@@ -1,0 +1,276 @@
+// Covariance-aware top-k routing with the score GEMM on the 5th-generation
+// tensor cores (AI Radio summary of PISA: score Score_{t,j}; gist.science
+// technical summary, section 2, covariance-aware routing).  For query block i
+// of a (batch, head):
+//   score_{i,j} = s qbar_i . kbar_j + ln(n_j + s ||qbar_i||_2 M_j)
+//   sel[i]      = the k largest scores, exact ties to the smaller j, ascending.
+// With M == nullptr the covariance term drops out (plain pooled routing).
+//
+// A CTA takes R query blocks of one (batch, head) and all nb key centroids:
+//   - the fp32 centroids arrive by TMA in stages of 128 blocks x 64 dims and
+//     are split in place into bf16 hi + lo (x = hi + lo + O(2^-18 |x|));
+//   - S^T = Kbar Qbar^T runs as tcgen05 MMAs with M = 128 key blocks, N = R
+//     query blocks, as hi.hi + hi.lo + lo.hi: an error of a few 1e-5 in the
+//     score for the largest workloads (|s qbar.kbar| ~ 40), well inside the
+//     1e-3 score gap the routing inputs keep between the k-th and (k+1)-th
+//     block;
+//   - each epilogue thread owns one key block (a TMEM lane): it reads the R
+//     scores of that block, adds the log term in fp32 and stores orderable
+//     keys [R][nb] in shared memory;
+//   - then every warp runs the per-row top-k (one warp per query block).
+// Warp roles (512 threads): 0-3 epilogue, 4-7 fp32 -> bf16 hi/lo conversion,
+// 8 TMA producer, 9 MMA issuer, all 16 warps for the top-k.
+#pragma once
+
+#include "select.cuh"
+#include "sm100.cuh"
+
+namespace pisa {
+
+constexpr int kSelTcThreads = 512;
+constexpr uint32_t kSelTcStage = 128u * 64u * 4u;  // 128 key blocks x 64 dims fp32 = bf16 hi + lo after the split
+
+template <int D, int R>
+struct SelectTcLayout {
+  static constexpr uint32_t kQ = R * D * 2u;  // Qbar hi (or lo): R rows x D bf16
+  __host__ __device__ static size_t keys_bytes(int nb) { return ((size_t)R * nb * 4 + 7) / 8 * 8; }
+  static size_t bytes(int ns, int nb) {
+    return 1024 + (size_t)ns * kSelTcStage + 2 * kQ + keys_bytes(nb) + R * 4 + (3 * (size_t)ns + 5) * 8 + 16;
+  }
+};
+
+// x[0..8) -> bf16 hi (RNE) and lo = bf16(x - hi), each as one 16-byte chunk.
+__device__ __forceinline__ void split_bf16x8(const float* x, uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const __nv_bfloat162 hv = __floats2bfloat162_rn(x[2 * e], x[2 * e + 1]);
+    const float2 hf = __bfloat1622float2(hv);
+    const __nv_bfloat162 lv = __floats2bfloat162_rn(x[2 * e] - hf.x, x[2 * e + 1] - hf.y);
+    h[e] = *reinterpret_cast<const uint32_t*>(&hv);
+    l[e] = *reinterpret_cast<const uint32_t*>(&lv);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Grid (ceil(nb / R), BH), kSelTcThreads threads, dynamic shared memory
+// SelectTcLayout<D, R>::bytes(ns, nb); ns >= 2 stages.
+// tmK: kbar fp32 [BH][nb][D], boxes of 32 dims x 128 blocks, 128-byte swizzle,
+// rows past nb read as zero.
+template <int D, int R>
+__global__ void __launch_bounds__(kSelTcThreads, 1)
+select_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const float* __restrict__ qbar,
+                    const float* __restrict__ M, int L, int B, int nb, int kk, int ns, float scale,
+                    int32_t* __restrict__ sel) {
+  using namespace sm100;
+  using Lay = SelectTcLayout<D, R>;
+  constexpr int NH = D / 64;                // stages per key tile
+  constexpr uint32_t STAGE = kSelTcStage;
+  constexpr uint32_t HALF = STAGE / 2;      // hi part, then lo part
+  constexpr uint32_t QB = R * 128u;         // one 64-dim block of Qbar hi (or lo)
+  constexpr uint32_t TCOLS = 2 * R < 32 ? 32 : 2 * R;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sStage = smem;                                   // [ns][STAGE]
+  uint8_t* sQh = smem + (size_t)ns * STAGE;                 // [NH][R][128 B]
+  uint8_t* sQl = sQh + Lay::kQ;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(sQl + Lay::kQ);  // [R][nb]
+  float* qn = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(keys) + Lay::keys_bytes(nb));  // [R]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(qn + R);
+  uint64_t* full = bars;              // [ns] fp32 stage landed
+  uint64_t* empty = bars + ns;        // [ns] stage read by the MMAs
+  uint64_t* conv = bars + 2 * ns;     // [ns] stage split into hi / lo
+  uint64_t* d_full = bars + 3 * ns;   // [2] scores of a key tile in TMEM
+  uint64_t* d_empty = d_full + 2;     // [2] scores read out of TMEM
+  uint64_t* mma_idle = d_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_idle + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int bh = blockIdx.y, i0 = blockIdx.x * R;
+  const int rows = min(R, nb - i0);
+  const int ntiles = (nb + 127) / 128;
+  const int nit = ntiles * NH;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ns; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&conv[s], 128);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&d_full[x], 1);
+      mbar_init(&d_empty[x], 128);
+    }
+    mbar_init(mma_idle, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, TCOLS);
+    tmem_relinquish();
+  }
+  // Qbar rows of this CTA as bf16 hi / lo, K-major with the 128-byte swizzle
+  // (16-byte chunk c of row r at position c ^ (r mod 8)); rows past nb are zero
+  for (int c = threadIdx.x; c < R * (D / 8); c += blockDim.x) {
+    const int r = c / (D / 8), c8 = c % (D / 8);
+    float x[8];
+    if (r < rows) {
+      load8(qbar + ((size_t)bh * nb + i0 + r) * D + 8 * c8, x);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] = 0.f;
+    }
+    uint4 hi, lo;
+    split_bf16x8(x, hi, lo);
+    const uint32_t off = (c8 / 8) * QB + r * 128u + (((c8 % 8) ^ (r & 7)) << 4);
+    *reinterpret_cast<uint4*>(sQh + off) = hi;
+    *reinterpret_cast<uint4*>(sQl + off) = lo;
+  }
+  fence_proxy_async_smem();
+  for (int r = warp; r < R; r += kSelTcThreads / 32) {
+    float t = 0.f;
+    if (r < rows) {
+      const float* q = qbar + ((size_t)bh * nb + i0 + r) * D;
+      for (int a = lane; a < D; a += 32) t = fmaf(q[a], q[a], t);
+    }
+    t = warp_sum(t);
+    if (lane == 0) qn[r] = sqrtf(t);
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ================================================================ producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmK);
+      int it = 0;
+      for (; it < nit; ++it) {
+        const int s = it % ns;
+        if (!mbar_wait(&empty[s], ((it / ns) & 1) ^ 1, abort)) break;
+        const int t = it / NH, h = it % NH;
+        mbar_expect_tx(&full[s], STAGE);
+        tma_load_3d(sStage + s * STAGE, &tmK, &full[s], h * 64, t * 128, bh);
+        tma_load_3d(sStage + s * STAGE + HALF, &tmK, &full[s], h * 64 + 32, t * 128, bh);
+      }
+      // the last load of each stage lands before the CTA can exit
+      for (int u = it > ns ? it - ns : 0; u < it; ++u) mbar_drain(&full[u % ns], (u / ns) & 1);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ================================================================ hi / lo split
+    // Thread r owns row r (key block t*128 + r) of the stage: it reads the row's
+    // 64 fp32 (two 128-byte rows, one per 32-dim box) and writes the row's 64
+    // bf16 hi into the first half and 64 bf16 lo into the second half, at the
+    // same byte offsets, so no thread writes where another one reads.
+    const int r = threadIdx.x - 128;
+    const uint32_t rsw = r & 7;
+    for (int it = 0; it < nit; ++it) {
+      const int s = it % ns;
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (it / ns) & 1, abort))) break;
+      uint8_t* st = sStage + s * STAGE;
+      float4 v[16];
+#pragma unroll
+      for (int b = 0; b < 2; ++b)
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          v[b * 8 + c] = *reinterpret_cast<const float4*>(st + b * HALF + r * 128u + ((c ^ rsw) << 4));
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) {
+        const float x[8] = {v[2 * c8].x, v[2 * c8].y, v[2 * c8].z, v[2 * c8].w,
+                            v[2 * c8 + 1].x, v[2 * c8 + 1].y, v[2 * c8 + 1].z, v[2 * c8 + 1].w};
+        uint4 hi, lo;
+        split_bf16x8(x, hi, lo);
+        const uint32_t off = r * 128u + ((c8 ^ rsw) << 4);
+        *reinterpret_cast<uint4*>(st + off) = hi;
+        *reinterpret_cast<uint4*>(st + HALF + off) = lo;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&conv[s]);
+    }
+  } else if (warp == 9) {
+    // ================================================================ MMA issuer
+    constexpr uint32_t idS = idesc_bf16(128, R, false, false);
+    const uint32_t stage0 = smem_u32(sStage), qh = smem_u32(sQh), ql = smem_u32(sQl);
+    bool ok = true;
+    int it = 0;
+    for (int t = 0; ok && t < ntiles; ++t) {
+      const int buf = t & 1;
+      if (t >= 2) {
+        if (!(ok = mbar_wait(&d_empty[buf], ((t >> 1) - 1) & 1, abort))) break;
+        fence_after_sync();
+      }
+      const uint32_t d = tmem + buf * R;
+      for (int h = 0; h < NH; ++h, ++it) {
+        const int s = it % ns;
+        if (!(ok = mbar_wait(&conv[s], (it / ns) & 1, abort))) break;
+        fence_after_sync();
+        const uint32_t ah = stage0 + s * STAGE, al = ah + HALF;
+        const uint32_t bhq = qh + h * QB, blq = ql + h * QB;
+#pragma unroll
+        for (int kk16 = 0; kk16 < 4; ++kk16) {
+          const uint64_t adh = desc_sw128(ah + kk16 * 32, 16, 1024), adl = desc_sw128(al + kk16 * 32, 16, 1024);
+          const uint64_t bdh = desc_sw128(bhq + kk16 * 32, 16, 1024), bdl = desc_sw128(blq + kk16 * 32, 16, 1024);
+          mma_ss_warp(d, adh, bdh, idS, (h > 0 || kk16 > 0) ? 1u : 0u);
+          mma_ss_warp(d, adh, bdl, idS, 1u);
+          mma_ss_warp(d, adl, bdh, idS, 1u);
+        }
+        mma_commit_warp(&empty[s]);
+      }
+      if (ok) mma_commit_warp(&d_full[buf]);
+    }
+    mma_commit_warp(mma_idle);
+    mbar_drain(mma_idle, 0);
+    __syncwarp();
+  } else if (warp < 4) {
+    // ================================================================ epilogue
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    for (int t = 0; t < ntiles; ++t) {
+      const int buf = t & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&d_full[buf], (t >> 1) & 1, abort))) break;
+      fence_after_sync();
+      uint32_t acc[R];
+      if constexpr (R == 32) {
+        tmem_ld32(lane_base + buf * R, acc);
+      } else {
+        tmem_ld16(lane_base + buf * R, acc);
+      }
+      tmem_wait_ld();
+      fence_before_sync();
+      mbar_arrive(&d_empty[buf]);
+      const int j = t * 128 + threadIdx.x;
+      if (j < nb) {
+        const float nj = (float)min(B, L - j * B);
+        const float mj = M != nullptr ? M[(size_t)bh * nb + j] : 0.f;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          if (r < rows)
+            keys[r * nb + j] =
+                orderable_key(fmaf(scale, __uint_as_float(acc[r]), __logf(fmaf(scale * qn[r], mj, nj))));
+        }
+      }
+    }
+  }
+
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  if (!*abort) {
+    // per-row selection, one warp per query block
+    for (int r = warp; r < rows; r += kSelTcThreads / 32)
+      topk_row_ascending(keys + r * nb, nb, kk, lane, sel + ((size_t)bh * nb + i0 + r) * kk);
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  if (warp == 9) tmem_dealloc(tmem, TCOLS);
+}
+
+}  // namespace pisa

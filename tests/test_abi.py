@@ -164,6 +164,20 @@ def test_routing_variant_entry_points_validate(lib):
         lib.PISA_ERR_INVALID_ARG
 
 
+def test_blockwise_entry_point_validates_before_any_cuda_call(lib):
+    raw = lib.raw_lib()
+    f = raw.pisa_attn_fwd_blockwise_with_sel
+    args = lambda H=FAKE, d=128, k=2, sel=FAKE, dt=lib.PISA_BF16: (
+        FAKE, FAKE, FAKE, FAKE, dt, 1, 1, 1000, d, 128, FAKE, FAKE, H, sel, k, None)
+    assert f(*args(H=None)) == lib.PISA_ERR_INVALID_ARG          # no block matrices
+    assert f(*args(H=MISALIGNED)) == lib.PISA_ERR_INVALID_ARG
+    assert f(*args(sel=None)) == lib.PISA_ERR_INVALID_ARG
+    assert f(*args(d=96)) == lib.PISA_ERR_UNSUPPORTED
+    assert f(*args(k=0)) == lib.PISA_ERR_INVALID_ARG
+    assert f(*args(k=9)) == lib.PISA_ERR_INVALID_ARG              # k > nb = 8
+    assert f(*args(dt=7)) == lib.PISA_ERR_INVALID_ARG
+
+
 def test_tuning_entry_points_validate_before_any_cuda_call(lib):
     raw = lib.raw_lib()
     t = lib._Tuning(0, 40, 0)  # select rows above 32

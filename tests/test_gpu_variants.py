@@ -13,7 +13,7 @@ import torch
 
 import oracle
 from workloads import small_config
-from parity_util import assert_output_close, assert_stat_close, inputs, to_device
+from parity_util import TOL, assert_output_close, assert_stat_close, inputs, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -114,3 +114,51 @@ def test_spectral_norm_equals_frobenius_for_rank_one_deviations(lib):
     frob = lib.cov_norm(kd, vd, B, stats[1], stats[2], stats[3]).cpu().numpy()
     torch.cuda.synchronize()
     np.testing.assert_allclose(spec, frob, rtol=1e-4)
+
+
+BLOCKWISE_CASES = [
+    small_config("blockwise_fp32", dtype="fp32", L=1000, d=64, block=64, heads=2, keep_ratio=0.25, seed=54),
+    small_config("blockwise_bf16_b128", L=2000, d=128, block=128, heads=2, keep_ratio=0.2, seed=55),
+    small_config("blockwise_bf16_b64", L=1100, d=128, block=64, heads=1, keep_ratio=0.1, seed=56),
+]
+
+
+@pytest.mark.parametrize("cfg", BLOCKWISE_CASES, ids=lambda c: c.name)
+def test_blockwise_first_order(lib, cfg):
+    """Each unselected block's own first-order term (pisa_attn_fwd_blockwise_with_sel)
+    against the oracle's blockwise variant on the GPU's selection, row by row;
+    and it is a different result from the hybrid term wherever H_j != Hbar."""
+    q, k, v = inputs(cfg, redraws={})
+    qd, kd, vd = (to_device(x, cfg.dtype) for x in (q, k, v))
+    B = cfg.block
+    kk = lib.keep_count(cfg.L, B, cfg.keep_ratio)
+    qbar, kbar, vsum, hbar = lib.block_stats(qd, kd, vd, B)
+    H = lib.block_first_order(kd, vd, B, kbar, vsum)
+    M = lib.cov_norm(kd, vd, B, kbar, vsum, hbar)
+    sel = lib.select(qbar, kbar, M, cfg.L, B, kk)
+    out = lib.attn_fwd_blockwise_with_sel(qd, kd, vd, B, kbar, vsum, H, sel)
+    hyb = lib.attn_fwd_with_sel(qd, kd, vd, B, kbar, vsum, hbar, sel)
+    torch.cuda.synchronize()
+    assert lib.device_status() == 0
+    s = 1.0 / math.sqrt(cfg.d)
+    checked = 0
+    for b in range(cfg.batch):
+        for h in range(cfg.heads):
+            qq, kk_, vv = (x[b, h].astype(np.float64) for x in (q, k, v))
+            qb, kb, vs, n = oracle.block_stats(qq, kk_, vv, B)
+            Hj = oracle.first_order_blocks(kk_, vv, B, kb)
+            ref = oracle.pisa_rows(qq, kk_, vv, B, sel[b, h].cpu().numpy(), kb, vs, n, oracle.hbar_mean(Hj),
+                                   np.arange(cfg.L), s, H_blocks=Hj)
+            got = out[b, h].float().cpu().numpy()
+            assert_output_close(got, ref, cfg.dtype, f"{cfg.name}[{b},{h}] blockwise")
+            # the variant is not the hybrid result in disguise: where the
+            # oracle's two results differ by more than 5x the tolerance, so do
+            # the GPU's (by more than the tolerance)
+            ref_hyb = oracle.pisa_rows(qq, kk_, vv, B, sel[b, h].cpu().numpy(), kb, vs, n, oracle.hbar_mean(Hj),
+                                       np.arange(cfg.L), s)
+            tol_abs = TOL[cfg.dtype][0]
+            if np.abs(ref - ref_hyb).max() > 5 * tol_abs:
+                checked += 1
+                gap = np.abs(got - hyb[b, h].float().cpu().numpy()).max()
+                assert gap > tol_abs, f"{cfg.name}[{b},{h}]: equals the hybrid output"
+    assert checked >= 1
