@@ -19,10 +19,12 @@ __device__ __forceinline__ uint32_t orderable_key(float f) {
 
 // The k largest of the nb keys kr[0..nb) (exact ties to the smaller index),
 // written to out[0..k) in ascending index order.  One warp per row, every lane
-// calls it.  An MSB-first bitwise search finds the k-th largest key (a 0 key
-// stands for "no block" and is never counted, since every candidate is >= 1);
-// then the keys above it and the first ties below it are compacted in index
-// order.  NR keys per lane are held in registers (nb <= 32 NR).
+// calls it.  An MSB-first bitwise search finds a threshold key: the k-th
+// largest key, or, as soon as exactly k keys reach a candidate, that
+// candidate (a 0 key stands for "no block" and is never counted, since every
+// candidate is >= 1); then the keys above the threshold and the first ties
+// at it are compacted in index order.  NR keys per lane are held in registers
+// (nb <= 32 NR).
 template <int NR>
 __device__ __forceinline__ uint32_t kth_largest_in_regs(const uint32_t* __restrict__ kr, int nb, int kk,
                                                        int lane) {
@@ -50,7 +52,12 @@ __device__ __forceinline__ uint32_t kth_largest_in_regs(const uint32_t* __restri
 #pragma unroll
     for (int m = 0; m < NR; ++m) cnt += (kv[m] >= cand);
     cnt = __reduce_add_sync(0xffffffffu, cnt);
-    if (cnt >= kk) prefix = cand;
+    if (cnt >= kk) {
+      prefix = cand;
+      // exactly k keys are >= cand: they are the top k, and cand separates
+      // them from the rest as well as the k-th key itself would
+      if (cnt == kk) break;
+    }
   }
   return prefix;
 }
@@ -73,7 +80,10 @@ __device__ __forceinline__ void topk_row_ascending(const uint32_t* __restrict__ 
       int cnt = 0;
       for (int j = lane; j < nb; j += 32) cnt += (kr[j] >= cand);
       cnt = __reduce_add_sync(0xffffffffu, cnt);
-      if (cnt >= kk) prefix = cand;
+      if (cnt >= kk) {
+        prefix = cand;
+        if (cnt == kk) break;
+      }
     }
     thr = prefix;
   }

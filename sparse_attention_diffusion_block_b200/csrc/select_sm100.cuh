@@ -18,8 +18,8 @@
 //     scores of that block, adds the log term in fp32 and stores orderable
 //     keys [R][nb] in shared memory;
 //   - then every warp runs the per-row top-k (one warp per query block).
-// Warp roles (512 threads): 0-3 epilogue, 4-7 fp32 -> bf16 hi/lo conversion,
-// 8 TMA producer, 9 MMA issuer, all 16 warps for the top-k.
+// Warp roles (512 threads): 0-3 epilogue, 4-7 and 12-15 fp32 -> bf16 hi/lo
+// split, 8 TMA producer, 9 MMA issuer, all 16 warps for the top-k.
 #pragma once
 
 #include "select.cuh"
@@ -102,7 +102,7 @@ select_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const float* __rest
     for (int s = 0; s < ns; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&conv[s], 128);
+      mbar_init(&conv[s], 256);
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&d_full[x], 1);
@@ -117,32 +117,29 @@ select_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const float* __rest
     tmem_relinquish();
   }
   // Qbar rows of this CTA as bf16 hi / lo, K-major with the 128-byte swizzle
-  // (16-byte chunk c of row r at position c ^ (r mod 8)); rows past nb are zero
-  for (int c = threadIdx.x; c < R * (D / 8); c += blockDim.x) {
+  // (16-byte chunk c of row r at position c ^ (r mod 8)); rows past nb are
+  // zero.  The D/8 threads of a row (consecutive lanes) also sum its squares.
+  static_assert(R * (D / 8) <= kSelTcThreads, "one 8-dim chunk per thread");
+  {
+    const int c = threadIdx.x;
     const int r = c / (D / 8), c8 = c % (D / 8);
-    float x[8];
-    if (r < rows) {
-      load8(qbar + ((size_t)bh * nb + i0 + r) * D + 8 * c8, x);
-    } else {
+    float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (c < R * (D / 8) && r < rows) load8(qbar + ((size_t)bh * nb + i0 + r) * D + 8 * c8, x);
+    float ss = 0.f;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) x[e] = 0.f;
+    for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+#pragma unroll
+    for (int o = 1; o < D / 8; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (c < R * (D / 8)) {
+      uint4 hi, lo;
+      split_bf16x8(x, hi, lo);
+      const uint32_t off = (c8 / 8) * QB + r * 128u + (((c8 % 8) ^ (r & 7)) << 4);
+      *reinterpret_cast<uint4*>(sQh + off) = hi;
+      *reinterpret_cast<uint4*>(sQl + off) = lo;
+      if (c8 == 0) qn[r] = sqrtf(ss);
     }
-    uint4 hi, lo;
-    split_bf16x8(x, hi, lo);
-    const uint32_t off = (c8 / 8) * QB + r * 128u + (((c8 % 8) ^ (r & 7)) << 4);
-    *reinterpret_cast<uint4*>(sQh + off) = hi;
-    *reinterpret_cast<uint4*>(sQl + off) = lo;
   }
   fence_proxy_async_smem();
-  for (int r = warp; r < R; r += kSelTcThreads / 32) {
-    float t = 0.f;
-    if (r < rows) {
-      const float* q = qbar + ((size_t)bh * nb + i0 + r) * D;
-      for (int a = lane; a < D; a += 32) t = fmaf(q[a], q[a], t);
-    }
-    t = warp_sum(t);
-    if (lane == 0) qn[r] = sqrtf(t);
-  }
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
@@ -164,31 +161,33 @@ select_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const float* __rest
       // the last load of each stage lands before the CTA can exit
       for (int u = it > ns ? it - ns : 0; u < it; ++u) mbar_drain(&full[u % ns], (u / ns) & 1);
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if ((warp >= 4 && warp < 8) || warp >= 12) {
     // ================================================================ hi / lo split
-    // Thread r owns row r (key block t*128 + r) of the stage: it reads the row's
-    // 64 fp32 (two 128-byte rows, one per 32-dim box) and writes the row's 64
-    // bf16 hi into the first half and 64 bf16 lo into the second half, at the
-    // same byte offsets, so no thread writes where another one reads.
-    const int r = threadIdx.x - 128;
+    // Eight warps, 16 rows each; lanes l and l + 16 share row r of the stage
+    // (key block t*128 + r): lane half b reads the row's 32 fp32 of box b and
+    // writes 32 bf16 hi (dims 32 b ..) into the first half of the stage and
+    // 32 bf16 lo into the second half, at the row's byte offsets.  Both halves
+    // of a row read before either writes (__syncwarp), and no other warp
+    // touches the row, so the split in place is safe.
+    const int cw = warp < 8 ? warp - 4 : warp - 8;  // 0..7
+    const int r = cw * 16 + (lane & 15), b = lane >> 4;
     const uint32_t rsw = r & 7;
     for (int it = 0; it < nit; ++it) {
       const int s = it % ns;
       if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (it / ns) & 1, abort))) break;
       uint8_t* st = sStage + s * STAGE;
-      float4 v[16];
+      float4 v[8];
 #pragma unroll
-      for (int b = 0; b < 2; ++b)
+      for (int c = 0; c < 8; ++c)
+        v[c] = *reinterpret_cast<const float4*>(st + b * HALF + r * 128u + ((c ^ rsw) << 4));
+      __syncwarp();
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          v[b * 8 + c] = *reinterpret_cast<const float4*>(st + b * HALF + r * 128u + ((c ^ rsw) << 4));
-#pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        const float x[8] = {v[2 * c8].x, v[2 * c8].y, v[2 * c8].z, v[2 * c8].w,
-                            v[2 * c8 + 1].x, v[2 * c8 + 1].y, v[2 * c8 + 1].z, v[2 * c8 + 1].w};
+      for (int c4 = 0; c4 < 4; ++c4) {
+        const float x[8] = {v[2 * c4].x, v[2 * c4].y, v[2 * c4].z, v[2 * c4].w,
+                            v[2 * c4 + 1].x, v[2 * c4 + 1].y, v[2 * c4 + 1].z, v[2 * c4 + 1].w};
         uint4 hi, lo;
         split_bf16x8(x, hi, lo);
-        const uint32_t off = r * 128u + ((c8 ^ rsw) << 4);
+        const uint32_t off = r * 128u + (((4 * b + c4) ^ rsw) << 4);
         *reinterpret_cast<uint4*>(st + off) = hi;
         *reinterpret_cast<uint4*>(st + HALF + off) = lo;
       }
@@ -234,6 +233,10 @@ select_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const float* __rest
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     for (int t = 0; t < ntiles; ++t) {
       const int buf = t & 1;
+      const int j = t * 128 + threadIdx.x;
+      // this key block's size and covariance norm, loaded before the wait
+      const float nj = j < nb ? (float)min(B, L - j * B) : 1.f;
+      const float mj = (M != nullptr && j < nb) ? M[(size_t)bh * nb + j] : 0.f;
       if (!__all_sync(0xffffffffu, mbar_wait(&d_full[buf], (t >> 1) & 1, abort))) break;
       fence_after_sync();
       uint32_t acc[R];
@@ -245,10 +248,7 @@ select_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const float* __rest
       tmem_wait_ld();
       fence_before_sync();
       mbar_arrive(&d_empty[buf]);
-      const int j = t * 128 + threadIdx.x;
       if (j < nb) {
-        const float nj = (float)min(B, L - j * B);
-        const float mj = M != nullptr ? M[(size_t)bh * nb + j] : 0.f;
 #pragma unroll
         for (int r = 0; r < R; ++r) {
           if (r < rows)

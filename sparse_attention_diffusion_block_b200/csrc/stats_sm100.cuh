@@ -25,9 +25,9 @@ struct StatsLayout {
   static constexpr uint32_t kTile = KB * D * 2u;        // one Q/K/V tile of a block
   static constexpr uint32_t kRing = kStatsStages * kTile;
   static constexpr uint32_t kOnes = 16 * KB * 2u;        // 16 x KB ones (K-major)
-  static constexpr uint32_t kSig = 2 * D * 4u;           // value-sum exchange, double buffered
+  static constexpr uint32_t kSig = 3 * D * 4u;           // value-sum exchange (2 buffers in the stats kernel, 3 in cov)
   static constexpr uint32_t kRed = 2 * 8 * 4u;           // cross-warp partials, double buffered
-  static constexpr uint32_t kBars = (2 * kStatsStages + 10) * 8u;
+  static constexpr uint32_t kBars = (2 * kStatsStages + 13) * 8u;
   static constexpr size_t bytes() { return 1024 + kRing + kOnes + kSig + kRed + kBars + 16; }
 };
 
@@ -265,7 +265,7 @@ cov_norm_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sRing = smem;
   float* sig = reinterpret_cast<float*>(smem + Lay::kRing + Lay::kOnes);  // [2][D]
-  float* red = sig + 2 * D;                                                // [2][8]
+  float* red = sig + Lay::kSig / 4;  // [2][8]
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sig) + Lay::kSig + Lay::kRed);
   uint64_t* full = bars;
   uint64_t* empty = bars + NS;
@@ -273,7 +273,8 @@ cov_norm_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
   uint64_t* d_free = d_full + 2;     // [2]
   uint64_t* mma_idle = d_free + 2;
   uint64_t* red_full = mma_idle + 1;  // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + 10);
+  uint64_t* vs_full = red_full + 2;   // [3] value sum of a block staged in sig
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NS + 13);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -286,6 +287,7 @@ cov_norm_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
+    for (int x = 0; x < 3; ++x) mbar_init(&vs_full[x], 128);
     mbar_init(&d_full[0], 1);
     mbar_init(&d_full[1], 1);
     mbar_init(&d_free[0], 128);
@@ -382,9 +384,16 @@ cov_norm_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
       const int j = j0 + jj;
       const size_t o = ((size_t)bh * nb + j) * D;
       const float kb = kbar[o + a];
-      // vsum_j is read by every thread straight from global memory (broadcast)
-      const float4* s4 = reinterpret_cast<const float4*>(vsum + o);
+      // every thread needs the whole vsum_j: staged in shared memory before
+      // the wait for H_j, so the load's latency hides behind it.  Three
+      // buffers: a thread starting block jj knows every epilogue thread has
+      // finished block jj - 3 (the MMA of jj - 1 waited for d_free of jj - 3).
+      const int vb = jj % 3;
+      sig[vb * D + a] = vsum[o + a];
+      mbar_arrive(&vs_full[vb]);
+      const float4* s4 = reinterpret_cast<const float4*>(sig + vb * D);
       if (!__all_sync(0xffffffffu, mbar_wait(&d_full[buf], (jj >> 1) & 1, abort))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&vs_full[vb], (jj / 3) & 1, abort))) break;
       fence_after_sync();
       float ss = 0.f;
 #pragma unroll
