@@ -561,6 +561,12 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           // register window, one per lane, refilled every 32 entries.
           int nvalid[G];
           bool all_whole = false;
+          // dead[h]: no row of this warp uses entry G u + h (its query block did
+          // not select it): that half's P is zero without any exp2 (64-token
+          // blocks only; a 128-token block is used by every row of the tile)
+          bool dead[G];
+#pragma unroll
+          for (int h = 0; h < G; ++h) dead[h] = false;
           if (exact) {
             if (((G * u) >> 5) != ent_win) {
               ent_win = (G * u) >> 5;
@@ -577,6 +583,7 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 if ((e >> (24 + g)) & 1) nvalid[h] = min(KB, a.L - j * KB);
               }
               whole = whole && nvalid[h] == KB;
+              if (G > 1) dead[h] = __all_sync(0xffffffffu, nvalid[h] == 0);
             }
             all_whole = __all_sync(0xffffffffu, whole);
           }
@@ -605,21 +612,26 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
               tmax = fmax3(fmaxf(t0, t1), t2, t3);
             } else {
               // masked columns (an absent half, or past a ragged tail) become
-              // -inf; four independent three-input max chains
+              // -inf; four independent three-input max chains; a dead half is
+              // skipped (its P is written as zero below)
               float t0 = -INFINITY, t1 = -INFINITY, t2 = -INFINITY, t3 = -INFINITY;
 #pragma unroll
-              for (int c = 0; c < 128; c += 8) {
-                float v[8];
+              for (int h = 0; h < G; ++h) {
+                if (dead[h]) continue;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                  const int cc = c + e;
-                  v[e] = (cc % KB) < nvalid[cc / KB] ? __uint_as_float(s[cc]) : -INFINITY;
-                  s[cc] = __float_as_uint(v[e]);
+                for (int c = h * KB; c < h * KB + KB; c += 8) {
+                  float v[8];
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) {
+                    const int cc = c + e;
+                    v[e] = (cc % KB) < nvalid[h] ? __uint_as_float(s[cc]) : -INFINITY;
+                    s[cc] = __float_as_uint(v[e]);
+                  }
+                  t0 = fmax3(t0, v[0], v[1]);
+                  t1 = fmax3(t1, v[2], v[3]);
+                  t2 = fmax3(t2, v[4], v[5]);
+                  t3 = fmax3(t3, v[6], v[7]);
                 }
-                t0 = fmax3(t0, v[0], v[1]);
-                t1 = fmax3(t1, v[2], v[3]);
-                t2 = fmax3(t2, v[4], v[5]);
-                t3 = fmax3(t3, v[6], v[7]);
               }
               tmax = fmax3(fmaxf(t0, t1), t2, t3);
             }
@@ -683,13 +695,21 @@ fused_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           const uint64_t c2x2 = f2_pack(c2, c2), nmu = f2_pack(-mu, -mu);
           uint64_t acc = 0;
 #pragma unroll
-          for (int c = 0; c < 128; c += 2) {
-            const uint64_t t = ffma2(f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), c2x2, nmu);
-            const float p0 = ex2(f2_lo(t));
-            const float p1 = ex2(f2_hi(t));
-            acc = fadd2(acc, f2_pack(p0, p1));
-            s[c >> 1] = pack_bf16x2(p0, p1);
-            if (c == 62) tmem_st32(sbase, s);  // keys 0..63 go out while 64..127 are computed
+          for (int hh = 0; hh < 2; ++hh) {
+            if (G > 1 && dead[hh * G / 2]) {
+#pragma unroll
+              for (int c = hh * 64; c < hh * 64 + 64; c += 2) s[c >> 1] = 0u;
+            } else {
+#pragma unroll
+              for (int c = hh * 64; c < hh * 64 + 64; c += 2) {
+                const uint64_t t = ffma2(f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), c2x2, nmu);
+                const float p0 = ex2(f2_lo(t));
+                const float p1 = ex2(f2_hi(t));
+                acc = fadd2(acc, f2_pack(p0, p1));
+                s[c >> 1] = pack_bf16x2(p0, p1);
+              }
+            }
+            if (hh == 0) tmem_st32(sbase, s);  // keys 0..63 go out while 64..127 are computed
           }
           const float sum = f2_lo(acc) + f2_hi(acc);
           if (exact) {

@@ -19,15 +19,16 @@ __device__ __forceinline__ uint32_t orderable_key(float f) {
 
 // The k largest of the nb keys kr[0..nb) (exact ties to the smaller index),
 // written to out[0..k) in ascending index order.  One warp per row, every lane
-// calls it.  An MSB-first bitwise search finds a threshold key: the k-th
-// largest key, or, as soon as exactly k keys reach a candidate, that
-// candidate (a 0 key stands for "no block" and is never counted, since every
-// candidate is >= 1); then the keys above the threshold and the first ties
-// at it are compacted in index order.  NR keys per lane are held in registers
-// (nb <= 32 NR).
+// calls it.  Lane l holds keys j = l + 32 m (m < NR, nb <= 32 NR) in registers.
+// An MSB-first bitwise search finds a threshold key: the k-th largest key, or,
+// as soon as exactly k keys reach a candidate, that candidate (a 0 key stands
+// for "no block" and is never counted, since every candidate is >= 1).  Then,
+// for m = 0, 1, ..., the warp takes the keys above the threshold and the
+// first of the keys equal to it, and places them with ballots and prefix
+// counts: indices come out ascending.
 template <int NR>
-__device__ __forceinline__ uint32_t kth_largest_in_regs(const uint32_t* __restrict__ kr, int nb, int kk,
-                                                       int lane) {
+__device__ __forceinline__ void topk_row_regs(const uint32_t* __restrict__ kr, int nb, int kk, int lane,
+                                              int32_t* __restrict__ out) {
   uint32_t kv[NR];
   uint32_t mx = 0u, mn = 0xffffffffu;
 #pragma unroll
@@ -42,52 +43,62 @@ __device__ __forceinline__ uint32_t kth_largest_in_regs(const uint32_t* __restri
   mx = __reduce_max_sync(0xffffffffu, mx);
   mn = __reduce_min_sync(0xffffffffu, mn);
   // the k-th largest lies in [mn, mx], so it shares their common high bits
+  uint32_t thr = mx;
   const uint32_t diff = mx ^ mn;
-  if (diff == 0u) return mx;
-  const int top = 31 - __clz(diff);
-  uint32_t prefix = (top == 31) ? 0u : (mx & ~((2u << top) - 1u));
-  for (int bit = top; bit >= 0; --bit) {
-    const uint32_t cand = prefix | (1u << bit);
-    int cnt = 0;
-#pragma unroll
-    for (int m = 0; m < NR; ++m) cnt += (kv[m] >= cand);
-    cnt = __reduce_add_sync(0xffffffffu, cnt);
-    if (cnt >= kk) {
-      prefix = cand;
-      // exactly k keys are >= cand: they are the top k, and cand separates
-      // them from the rest as well as the k-th key itself would
-      if (cnt == kk) break;
-    }
-  }
-  return prefix;
-}
-
-__device__ __forceinline__ void topk_row_ascending(const uint32_t* __restrict__ kr, int nb, int kk, int lane,
-                                                   int32_t* __restrict__ out) {
-  uint32_t thr;  // k-th largest key
-  if (nb <= 256) {
-    thr = kth_largest_in_regs<8>(kr, nb, kk, lane);
-  } else if (nb <= 512) {
-    thr = kth_largest_in_regs<16>(kr, nb, kk, lane);
-  } else if (nb <= 768) {
-    thr = kth_largest_in_regs<24>(kr, nb, kk, lane);
-  } else if (nb <= 1024) {
-    thr = kth_largest_in_regs<32>(kr, nb, kk, lane);
-  } else {
-    uint32_t prefix = 0;
-    for (int bit = 31; bit >= 0; --bit) {
+  if (diff != 0u) {
+    const int top = 31 - __clz(diff);
+    uint32_t prefix = (top == 31) ? 0u : (mx & ~((2u << top) - 1u));
+    for (int bit = top; bit >= 0; --bit) {
       const uint32_t cand = prefix | (1u << bit);
-      int cnt = 0;
-      for (int j = lane; j < nb; j += 32) cnt += (kr[j] >= cand);
-      cnt = __reduce_add_sync(0xffffffffu, cnt);
+      // four independent partial counts: a short dependency chain to the reduce
+      int c4[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int m = 0; m < NR; ++m) c4[m & 3] += (kv[m] >= cand);
+      const int cnt = __reduce_add_sync(0xffffffffu, (c4[0] + c4[1]) + (c4[2] + c4[3]));
       if (cnt >= kk) {
         prefix = cand;
+        // exactly k keys are >= cand: they are the top k, and cand separates
+        // them from the rest as well as the k-th key itself would
         if (cnt == kk) break;
       }
     }
     thr = prefix;
   }
-  const int C = (nb + 31) / 32;  // contiguous chunk of indices per lane
+  int gt = 0;
+#pragma unroll
+  for (int m = 0; m < NR; ++m) gt += (kv[m] > thr);
+  int need = kk - __reduce_add_sync(0xffffffffu, gt);  // ties taken, lowest indices first
+  const uint32_t below = (1u << lane) - 1u;
+  int base = 0;
+#pragma unroll
+  for (int m = 0; m < NR; ++m) {
+    const bool eq = kv[m] == thr;
+    const uint32_t be = __ballot_sync(0xffffffffu, eq);
+    const bool take = kv[m] > thr || (eq && __popc(be & below) < need);
+    const uint32_t bt = __ballot_sync(0xffffffffu, take);
+    if (take) out[base + __popc(bt & below)] = lane + 32 * m;
+    base += __popc(bt);
+    need -= min(__popc(be), max(need, 0));
+  }
+}
+
+// The same for any nb, keys read from shared memory: lane l takes the
+// contiguous indices [l C, l C + C).
+__device__ __forceinline__ void topk_row_smem(const uint32_t* __restrict__ kr, int nb, int kk, int lane,
+                                              int32_t* __restrict__ out) {
+  uint32_t prefix = 0;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = prefix | (1u << bit);
+    int cnt = 0;
+    for (int j = lane; j < nb; j += 32) cnt += (kr[j] >= cand);
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
+    if (cnt >= kk) {
+      prefix = cand;
+      if (cnt == kk) break;
+    }
+  }
+  const uint32_t thr = prefix;
+  const int C = (nb + 31) / 32;
   const int jb = min(nb, lane * C), je = min(nb, jb + C);
   int n_gt = 0, n_eq = 0;
   for (int j = jb; j < je; ++j) {
@@ -122,6 +133,21 @@ __device__ __forceinline__ void topk_row_ascending(const uint32_t* __restrict__ 
       ++eq_taken;
     }
     if (take) out[pos++] = j;
+  }
+}
+
+__device__ __forceinline__ void topk_row_ascending(const uint32_t* __restrict__ kr, int nb, int kk, int lane,
+                                                   int32_t* __restrict__ out) {
+  if (nb <= 256) {
+    topk_row_regs<8>(kr, nb, kk, lane, out);
+  } else if (nb <= 512) {
+    topk_row_regs<16>(kr, nb, kk, lane, out);
+  } else if (nb <= 768) {
+    topk_row_regs<24>(kr, nb, kk, lane, out);
+  } else if (nb <= 1024) {
+    topk_row_regs<32>(kr, nb, kk, lane, out);
+  } else {
+    topk_row_smem(kr, nb, kk, lane, out);
   }
 }
 

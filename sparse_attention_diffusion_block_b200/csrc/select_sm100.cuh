@@ -231,6 +231,9 @@ select_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const float* __rest
   } else if (warp < 4) {
     // ================================================================ epilogue
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    float sq[R];  // s ||qbar_r||, in registers for the whole loop
+#pragma unroll
+    for (int r = 0; r < R; ++r) sq[r] = scale * qn[r];
     for (int t = 0; t < ntiles; ++t) {
       const int buf = t & 1;
       const int j = t * 128 + threadIdx.x;
@@ -253,7 +256,7 @@ select_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const float* __rest
         for (int r = 0; r < R; ++r) {
           if (r < rows)
             keys[r * nb + j] =
-                orderable_key(fmaf(scale, __uint_as_float(acc[r]), __logf(fmaf(scale * qn[r], mj, nj))));
+                orderable_key(fmaf(scale, __uint_as_float(acc[r]), __logf(fmaf(sq[r], mj, nj))));
         }
       }
     }
