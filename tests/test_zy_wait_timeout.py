@@ -1,12 +1,14 @@
 """Bounded device waits that run out, and the unwind after them.
 
 Every mbarrier wait between the warps of the tensor-core kernels (statistics,
-covariance norm, fused attention) is bounded.  A wait that runs out records
+covariance norm, routing, fused attention) is bounded.  A wait that runs out records
 PISA_ERR_TIMEOUT in the device error word, the CTA lets the copies and MMAs it
 already issued complete, frees its tensor memory and exits.  Here the limit is
 set to 1 ns through pisa_set_wait_limit, so the first wait that has to spin
 gives up: nothing faults or hangs, the host reads the status, and the same
-process then runs a normal forward that matches the oracle.
+process then runs a normal forward that matches the oracle.  The routing call
+runs on valid statistics; its selections are then undefined (the timed-out
+CTAs skip the top-k), and the fused call uses the selections computed before.
 
 Collected after the other GPU tests (and before the no-allocation entry
 point's file), so that a run stopping at the first failure has run them.
@@ -46,6 +48,7 @@ def test_short_wait_limit_times_out_each_kernel_then_context_stays_usable(lib):
     stages = {
         "statistics": lambda: lib.block_stats(qd, kd, vd, B),
         "covariance norm": lambda: lib.cov_norm(kd, vd, B, kbar, vsum, hbar),
+        "routing": lambda: lib.select(qbar, kbar, M, CFG.L, B, kk),
         "fused attention": lambda: lib.attn_fwd_with_sel(qd, kd, vd, B, kbar, vsum, hbar, sel),
     }
     try:
