@@ -168,3 +168,36 @@ def test_named_workload(lib, name):
         rows = np.concatenate([np.arange(i * B, min((i + 1) * B, cfg.L)) for i in blocks])
         r = oracle_head(q[b, h], k[b, h], v[b, h], B, kk, rows=rows)
         assert_output_close(out_np[b, h, rows], r["out"], cfg.dtype, f"{name} [{b},{h}]")
+
+
+# ---------------------------------------------------------------- routing configurations for many blocks
+
+MANY_BLOCKS = [
+    # 1250 blocks: the tensor-core routing kernel runs 16 query blocks per CTA
+    small_config("route_r16", L=80000, d=128, block=64, heads=1, keep_ratio=0.02, seed=61),
+    # 2500 blocks: past its shared memory, the CUDA-core routing kernel takes over
+    small_config("route_cuda_cores", L=160000, d=128, block=64, heads=1, keep_ratio=0.01, seed=62),
+]
+
+
+@pytest.mark.parametrize("cfg", MANY_BLOCKS, ids=lambda c: c.name)
+def test_routing_for_many_blocks(lib, cfg):
+    """S_i bit for bit against the oracle, M_j and sampled output rows, where
+    nb is large enough to change the routing kernel's configuration."""
+    q, k, v = inputs(cfg)
+    kk = lib.keep_count(cfg.L, cfg.block, cfg.keep_ratio)
+    qd, kd, vd = (to_device(x, cfg.dtype) for x in (q, k, v))
+    B = cfg.block
+    qbar, kbar, vsum, hbar = lib.block_stats(qd, kd, vd, B)
+    M = lib.cov_norm(kd, vd, B, kbar, vsum, hbar)
+    sel = lib.select(qbar, kbar, M, cfg.L, B, kk)
+    out = lib.attn_fwd(qd, kd, vd, B, cfg.keep_ratio)
+    torch.cuda.synchronize()
+    assert lib.device_status() == 0
+    r = oracle_routing(q[0, 0], k[0, 0], v[0, 0], B, kk)
+    np.testing.assert_array_equal(sel[0, 0].cpu().numpy(), r["sel"], err_msg=f"{cfg.name} S_i")
+    assert np.abs(M[0, 0].cpu().numpy() - r["M"]).max() <= 1e-5 * max(r["H_scale"], 1e-30)
+    blocks = _sample_blocks(cfg.nb, np.random.default_rng(cfg.seed), n=4)
+    rows = np.concatenate([np.arange(i * B, min((i + 1) * B, cfg.L)) for i in blocks])
+    ro = oracle_head(q[0, 0], k[0, 0], v[0, 0], B, kk, rows=rows)
+    assert_output_close(out[0, 0, rows].float().cpu().numpy(), ro["out"], cfg.dtype, cfg.name)
