@@ -7,8 +7,11 @@
 // With M == nullptr the covariance term drops out (plain pooled routing).
 //
 // A CTA takes R query blocks of one (batch, head) and all nb key centroids:
-//   - the fp32 centroids arrive by TMA in stages of 128 blocks x 64 dims and
-//     are split in place into bf16 hi + lo (x = hi + lo + O(2^-18 |x|));
+//   - the fp32 centroids arrive by TMA in stages of 128 blocks x 64 dims; the
+//     split warps read a stage, hand it back to the producer and write it as
+//     bf16 hi + lo (x = hi + lo + O(2^-18 |x|)) into tensor memory, where the
+//     MMAs read it as their A operand (shared memory carries only the fp32
+//     stages and Qbar, no split copy of the centroids);
 //   - S^T = Kbar Qbar^T runs as tcgen05 MMAs with M = 128 key blocks, N = R
 //     query blocks, as hi.hi + hi.lo + lo.hi: an error of a few 1e-5 in the
 //     score for the largest workloads (|s qbar.kbar| ~ 40), well inside the
@@ -20,6 +23,8 @@
 //   - then every warp runs the per-row top-k (one warp per query block).
 // Warp roles (512 threads): 0-3 epilogue, 4-7 and 12-15 fp32 -> bf16 hi/lo
 // split, 8 TMA producer, 9 MMA issuer, all 16 warps for the top-k.
+// TMEM columns: [0, 2R) the scores of two key tiles; [128, 256) and [256, 384)
+// the hi (first 64 columns) and lo (last 64) centroids of two key tiles.
 #pragma once
 
 #include "select.cuh"
@@ -28,14 +33,14 @@
 namespace pisa {
 
 constexpr int kSelTcThreads = 512;
-constexpr uint32_t kSelTcStage = 128u * 64u * 4u;  // 128 key blocks x 64 dims fp32 = bf16 hi + lo after the split
+constexpr uint32_t kSelTcStage = 128u * 64u * 4u;  // 128 key blocks x 64 dims fp32
 
 template <int D, int R>
 struct SelectTcLayout {
   static constexpr uint32_t kQ = R * D * 2u;  // Qbar hi (or lo): R rows x D bf16
   __host__ __device__ static size_t keys_bytes(int nb) { return ((size_t)R * nb * 4 + 7) / 8 * 8; }
   static size_t bytes(int ns, int nb) {
-    return 1024 + (size_t)ns * kSelTcStage + 2 * kQ + keys_bytes(nb) + R * 4 + (3 * (size_t)ns + 5) * 8 + 16;
+    return 1024 + (size_t)ns * kSelTcStage + 2 * kQ + keys_bytes(nb) + R * 4 + (2 * (size_t)ns + 9) * 8 + 16;
   }
 };
 
@@ -71,9 +76,11 @@ select_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const float* __rest
   using Lay = SelectTcLayout<D, R>;
   constexpr int NH = D / 64;                // stages per key tile
   constexpr uint32_t STAGE = kSelTcStage;
-  constexpr uint32_t HALF = STAGE / 2;      // hi part, then lo part
+  constexpr uint32_t HALF = STAGE / 2;      // the stage's two 32-dim boxes
   constexpr uint32_t QB = R * 128u;         // one 64-dim block of Qbar hi (or lo)
-  constexpr uint32_t TCOLS = 2 * R < 32 ? 32 : 2 * R;
+  constexpr uint32_t TCOLS = 512;
+  constexpr uint32_t ACOL = 128;            // hi / lo centroid buffers in TMEM
+  static_assert(2 * R <= ACOL, "score buffers below the centroid buffers");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -84,9 +91,10 @@ select_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const float* __rest
   float* qn = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(keys) + Lay::keys_bytes(nb));  // [R]
   uint64_t* bars = reinterpret_cast<uint64_t*>(qn + R);
   uint64_t* full = bars;              // [ns] fp32 stage landed
-  uint64_t* empty = bars + ns;        // [ns] stage read by the MMAs
-  uint64_t* conv = bars + 2 * ns;     // [ns] stage split into hi / lo
-  uint64_t* d_full = bars + 3 * ns;   // [2] scores of a key tile in TMEM
+  uint64_t* empty = bars + ns;        // [ns] stage read by the split warps
+  uint64_t* a_full = bars + 2 * ns;   // [2] hi / lo centroids of a key tile in TMEM
+  uint64_t* a_empty = a_full + 2;     // [2] ... read by the MMAs
+  uint64_t* d_full = a_empty + 2;     // [2] scores of a key tile in TMEM
   uint64_t* d_empty = d_full + 2;     // [2] scores read out of TMEM
   uint64_t* mma_idle = d_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_idle + 1);
@@ -101,10 +109,11 @@ select_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const float* __rest
   if (threadIdx.x == 0) {
     for (int s = 0; s < ns; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-      mbar_init(&conv[s], 256);
+      mbar_init(&empty[s], 4);  // the four split warps of the stage's half
     }
     for (int x = 0; x < 2; ++x) {
+      mbar_init(&a_full[x], 4 * NH);
+      mbar_init(&a_empty[x], 1);
       mbar_init(&d_full[x], 1);
       mbar_init(&d_empty[x], 128);
     }
@@ -162,68 +171,77 @@ select_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const float* __rest
       for (int u = it > ns ? it - ns : 0; u < it; ++u) mbar_drain(&full[u % ns], (u / ns) & 1);
     }
   } else if ((warp >= 4 && warp < 8) || warp >= 12) {
-    // ================================================================ hi / lo split
-    // Eight warps, 16 rows each; lanes l and l + 16 share row r of the stage
-    // (key block t*128 + r): lane half b reads the row's 32 fp32 of box b and
-    // writes 32 bf16 hi (dims 32 b ..) into the first half of the stage and
-    // 32 bf16 lo into the second half, at the row's byte offsets.  Both halves
-    // of a row read before either writes (__syncwarp), and no other warp
-    // touches the row, so the split in place is safe.
-    const int cw = warp < 8 ? warp - 4 : warp - 8;  // 0..7
-    const int r = cw * 16 + (lane & 15), b = lane >> 4;
+    // ================================================================ hi / lo split into TMEM
+    // Warp w owns TMEM lane quarter q = w % 4, i.e. key blocks 32 q + lane of
+    // each tile, and the stages of dim half c (warps 4-7: dims 0-63, warps
+    // 12-15: dims 64-127).  Lane l reads its row's 64 fp32 from the stage,
+    // the warp hands the stage back to the producer, and the row goes to
+    // TMEM as 32 columns of bf16x2 hi and 32 of lo (dims 2w, 2w+1 in column
+    // w of the half).
+    const int q = warp % 4, c = warp < 8 ? 0 : 1;
+    const int r = 32 * q + lane;
     const uint32_t rsw = r & 7;
-    for (int it = 0; it < nit; ++it) {
-      const int s = it % ns;
+    const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
+    for (int it = c; c < NH && it < nit; it += NH) {
+      const int s = it % ns, t = it / NH, buf = t & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (it / ns) & 1, abort))) break;
-      uint8_t* st = sStage + s * STAGE;
-      float4 v[8];
+      const uint8_t* st = sStage + s * STAGE;
+      float4 v[16];  // v[8 b + k]: chunk k of box b (dims 32 b + 4 k ..)
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        v[c] = *reinterpret_cast<const float4*>(st + b * HALF + r * 128u + ((c ^ rsw) << 4));
+      for (int k = 0; k < 16; ++k)
+        v[k] = *reinterpret_cast<const float4*>(st + (k / 8) * HALF + r * 128u + (((k % 8) ^ rsw) << 4));
       __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      // the MMAs of tile t - 2 have read this TMEM buffer
+      if (t >= 2 && !__all_sync(0xffffffffu, mbar_wait(&a_empty[buf], ((t >> 1) - 1) & 1, abort))) break;
+      const uint32_t ab = tmem + lane_off + ACOL + buf * 128 + c * 32;
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        const float x[8] = {v[2 * c4].x, v[2 * c4].y, v[2 * c4].z, v[2 * c4].w,
-                            v[2 * c4 + 1].x, v[2 * c4 + 1].y, v[2 * c4 + 1].z, v[2 * c4 + 1].w};
-        uint4 hi, lo;
-        split_bf16x8(x, hi, lo);
-        const uint32_t off = r * 128u + (((4 * b + c4) ^ rsw) << 4);
-        *reinterpret_cast<uint4*>(st + off) = hi;
-        *reinterpret_cast<uint4*>(st + HALF + off) = lo;
+      for (int b = 0; b < 2; ++b) {
+        uint32_t hw[16], lw[16];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const float4 x0 = v[8 * b + 2 * g], x1 = v[8 * b + 2 * g + 1];
+          const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+          uint4 hi, lo;
+          split_bf16x8(x, hi, lo);
+          hw[4 * g] = hi.x, hw[4 * g + 1] = hi.y, hw[4 * g + 2] = hi.z, hw[4 * g + 3] = hi.w;
+          lw[4 * g] = lo.x, lw[4 * g + 1] = lo.y, lw[4 * g + 2] = lo.z, lw[4 * g + 3] = lo.w;
+        }
+        tmem_st16(ab + 16 * b, hw);
+        tmem_st16(ab + 64 + 16 * b, lw);
       }
-      fence_proxy_async_smem();
-      mbar_arrive(&conv[s]);
+      tmem_wait_st();
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&a_full[buf]);
     }
   } else if (warp == 9) {
     // ================================================================ MMA issuer
+    // A (centroid hi / lo) from TMEM, B (Qbar hi / lo) from shared memory; the
+    // three products of each 16-dim step in the same order as always.
     constexpr uint32_t idS = idesc_bf16(128, R, false, false);
-    const uint32_t stage0 = smem_u32(sStage), qh = smem_u32(sQh), ql = smem_u32(sQl);
+    const uint32_t qh = smem_u32(sQh), ql = smem_u32(sQl);
     bool ok = true;
-    int it = 0;
     for (int t = 0; ok && t < ntiles; ++t) {
       const int buf = t & 1;
-      if (t >= 2) {
-        if (!(ok = mbar_wait(&d_empty[buf], ((t >> 1) - 1) & 1, abort))) break;
-        fence_after_sync();
-      }
+      if (!(ok = mbar_wait(&a_full[buf], (t >> 1) & 1, abort))) break;
+      if (t >= 2 && !(ok = mbar_wait(&d_empty[buf], ((t >> 1) - 1) & 1, abort))) break;
+      fence_after_sync();
       const uint32_t d = tmem + buf * R;
-      for (int h = 0; h < NH; ++h, ++it) {
-        const int s = it % ns;
-        if (!(ok = mbar_wait(&conv[s], (it / ns) & 1, abort))) break;
-        fence_after_sync();
-        const uint32_t ah = stage0 + s * STAGE, al = ah + HALF;
+      const uint32_t ah = tmem + ACOL + buf * 128, al = ah + 64;
+      for (int h = 0; h < NH; ++h) {
         const uint32_t bhq = qh + h * QB, blq = ql + h * QB;
 #pragma unroll
         for (int kk16 = 0; kk16 < 4; ++kk16) {
-          const uint64_t adh = desc_sw128(ah + kk16 * 32, 16, 1024), adl = desc_sw128(al + kk16 * 32, 16, 1024);
+          const uint32_t ac = (h * 4 + kk16) * 8;
           const uint64_t bdh = desc_sw128(bhq + kk16 * 32, 16, 1024), bdl = desc_sw128(blq + kk16 * 32, 16, 1024);
-          mma_ss_warp(d, adh, bdh, idS, (h > 0 || kk16 > 0) ? 1u : 0u);
-          mma_ss_warp(d, adh, bdl, idS, 1u);
-          mma_ss_warp(d, adl, bdh, idS, 1u);
+          mma_ts_warp(d, ah + ac, bdh, idS, (h > 0 || kk16 > 0) ? 1u : 0u);
+          mma_ts_warp(d, ah + ac, bdl, idS, 1u);
+          mma_ts_warp(d, al + ac, bdh, idS, 1u);
         }
-        mma_commit_warp(&empty[s]);
       }
-      if (ok) mma_commit_warp(&d_full[buf]);
+      mma_commit_warp(&d_full[buf]);
+      mma_commit_warp(&a_empty[buf]);
     }
     mma_commit_warp(mma_idle);
     mbar_drain(mma_idle, 0);
