@@ -17,14 +17,33 @@ __device__ __forceinline__ uint32_t orderable_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Count of the warp's keys kv (NR per lane) that are >= c: four independent
+// partial counts, a short dependency chain to the reduce.
+template <int NR>
+__device__ __forceinline__ int count_at_least(const uint32_t (&kv)[NR], uint32_t c) {
+  int c4[4] = {0, 0, 0, 0};
+#pragma unroll
+  for (int m = 0; m < NR; ++m) c4[m & 3] += (kv[m] >= c);
+  return __reduce_add_sync(0xffffffffu, (c4[0] + c4[1]) + (c4[2] + c4[3]));
+}
+
 // The k largest of the nb keys kr[0..nb) (exact ties to the smaller index),
 // written to out[0..k) in ascending index order.  One warp per row, every lane
 // calls it.  Lane l holds keys j = l + 32 m (m < NR, nb <= 32 NR) in registers.
-// An MSB-first bitwise search finds a threshold key: the k-th largest key, or,
-// as soon as exactly k keys reach a candidate, that candidate (a 0 key stands
-// for "no block" and is never counted, since every candidate is >= 1).  Then,
-// for m = 0, 1, ..., the warp takes the keys above the threshold and the
-// first of the keys equal to it, and places them with ballots and prefix
+// A search over key values finds a threshold: a key value t with exactly k
+// keys >= t (any such t separates the top k), or else the k-th largest key
+// itself.  A 0 key stands for "no block" and is never counted: every
+// candidate is above the smallest real key.
+//   - NR >= 16: a bracket lo < hi with count(>= lo) >= k > count(>= hi); each
+//     round tries the candidate that linear interpolation of the two counts
+//     points to, and a round that fails to halve the bracket makes the next
+//     one bisect, so the search ends within 64 rounds (~9-10 on the video
+//     workloads, against ~12-17 for the bitwise search);
+//   - NR < 16: MSB-first bitwise search below the common high bits of the
+//     largest and smallest key (a round is cheap enough that the extra
+//     interpolation arithmetic would not pay).
+// Then, for m = 0, 1, ..., the warp takes the keys above the threshold and
+// the first of the keys equal to it, and places them with ballots and prefix
 // counts: indices come out ascending.
 template <int NR>
 __device__ __forceinline__ void topk_row_regs(const uint32_t* __restrict__ kr, int nb, int kk, int lane,
@@ -42,27 +61,58 @@ __device__ __forceinline__ void topk_row_regs(const uint32_t* __restrict__ kr, i
   }
   mx = __reduce_max_sync(0xffffffffu, mx);
   mn = __reduce_min_sync(0xffffffffu, mn);
-  // the k-th largest lies in [mn, mx], so it shares their common high bits
-  uint32_t thr = mx;
-  const uint32_t diff = mx ^ mn;
-  if (diff != 0u) {
-    const int top = 31 - __clz(diff);
-    uint32_t prefix = (top == 31) ? 0u : (mx & ~((2u << top) - 1u));
-    for (int bit = top; bit >= 0; --bit) {
-      const uint32_t cand = prefix | (1u << bit);
-      // four independent partial counts: a short dependency chain to the reduce
-      int c4[4] = {0, 0, 0, 0};
-#pragma unroll
-      for (int m = 0; m < NR; ++m) c4[m & 3] += (kv[m] >= cand);
-      const int cnt = __reduce_add_sync(0xffffffffu, (c4[0] + c4[1]) + (c4[2] + c4[3]));
-      if (cnt >= kk) {
-        prefix = cand;
-        // exactly k keys are >= cand: they are the top k, and cand separates
-        // them from the rest as well as the k-th key itself would
-        if (cnt == kk) break;
+  uint32_t thr = mn;  // k == nb: every key
+  if (kk < nb) {
+    if constexpr (NR >= 16) {
+      uint64_t lo = mn, hi = (uint64_t)mx + 1u;  // count(>= lo) = nb, count(>= hi) = 0
+      int clo = nb, chi = 0;
+      bool bisect = false, found = false;
+      while (hi - lo > 1u) {
+        const uint64_t w = hi - lo;
+        uint64_t cand;
+        if (bisect) {
+          cand = lo + w / 2u;
+        } else {
+          const float f = (float)(clo - kk) / (float)(clo - chi);
+          cand = lo + (uint64_t)(f * (float)w);
+          cand = cand < lo + 1u ? lo + 1u : (cand > hi - 1u ? hi - 1u : cand);
+        }
+        const int cnt = count_at_least(kv, (uint32_t)cand);
+        if (cnt == kk) {
+          thr = (uint32_t)cand;
+          found = true;
+          break;
+        }
+        if (cnt > kk) {
+          lo = cand;
+          clo = cnt;
+        } else {
+          hi = cand;
+          chi = cnt;
+        }
+        bisect = (hi - lo) > w / 2u;
+      }
+      if (!found) thr = (uint32_t)lo;  // the k-th largest key (ties at it)
+    } else {
+      // the k-th largest lies in [mn, mx], so it shares their common high bits
+      thr = mx;
+      const uint32_t diff = mx ^ mn;
+      if (diff != 0u) {
+        const int top = 31 - __clz(diff);
+        uint32_t prefix = (top == 31) ? 0u : (mx & ~((2u << top) - 1u));
+        for (int bit = top; bit >= 0; --bit) {
+          const uint32_t cand = prefix | (1u << bit);
+          const int cnt = count_at_least(kv, cand);
+          if (cnt >= kk) {
+            prefix = cand;
+            // exactly k keys are >= cand: they are the top k, and cand
+            // separates them from the rest as well as the k-th key would
+            if (cnt == kk) break;
+          }
+        }
+        thr = prefix;
       }
     }
-    thr = prefix;
   }
   int gt = 0;
 #pragma unroll
@@ -138,12 +188,21 @@ __device__ __forceinline__ void topk_row_smem(const uint32_t* __restrict__ kr, i
 
 __device__ __forceinline__ void topk_row_ascending(const uint32_t* __restrict__ kr, int nb, int kk, int lane,
                                                    int32_t* __restrict__ out) {
-  if (nb <= 256) {
+  // as few key registers per lane as the row needs (a multiple of four)
+  if (nb <= 128) {
+    topk_row_regs<4>(kr, nb, kk, lane, out);
+  } else if (nb <= 256) {
     topk_row_regs<8>(kr, nb, kk, lane, out);
+  } else if (nb <= 384) {
+    topk_row_regs<12>(kr, nb, kk, lane, out);
   } else if (nb <= 512) {
     topk_row_regs<16>(kr, nb, kk, lane, out);
+  } else if (nb <= 640) {
+    topk_row_regs<20>(kr, nb, kk, lane, out);
   } else if (nb <= 768) {
     topk_row_regs<24>(kr, nb, kk, lane, out);
+  } else if (nb <= 896) {
+    topk_row_regs<28>(kr, nb, kk, lane, out);
   } else if (nb <= 1024) {
     topk_row_regs<32>(kr, nb, kk, lane, out);
   } else {
