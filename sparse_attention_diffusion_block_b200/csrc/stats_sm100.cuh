@@ -395,7 +395,8 @@ cov_norm_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
       if (!__all_sync(0xffffffffu, mbar_wait(&d_full[buf], (jj >> 1) & 1, abort))) break;
       if (!__all_sync(0xffffffffu, mbar_wait(&vs_full[vb], (jj / 3) & 1, abort))) break;
       fence_after_sync();
-      float ss = 0.f;
+      // four independent partial sums (columns b mod 4), added in a fixed order
+      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t h[32];
@@ -408,12 +409,13 @@ cov_norm_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
           const float d1 = __uint_as_float(h[e + 1]) - fmaf(kb, w.y, hb[ch * 32 + e + 1]);
           const float d2 = __uint_as_float(h[e + 2]) - fmaf(kb, w.z, hb[ch * 32 + e + 2]);
           const float d3 = __uint_as_float(h[e + 3]) - fmaf(kb, w.w, hb[ch * 32 + e + 3]);
-          ss = fmaf(d0, d0, ss);
-          ss = fmaf(d1, d1, ss);
-          ss = fmaf(d2, d2, ss);
-          ss = fmaf(d3, d3, ss);
+          s0 = fmaf(d0, d0, s0);
+          s1 = fmaf(d1, d1, s1);
+          s2 = fmaf(d2, d2, s2);
+          s3 = fmaf(d3, d3, s3);
         }
       }
+      float ss = (s0 + s1) + (s2 + s3);
       // fixed-order reduction over the four warps; red[buf] is rewritten two
       // blocks later, after thread 0 (which reads it) has arrived on d_free.
       ss = warp_sum(ss);
