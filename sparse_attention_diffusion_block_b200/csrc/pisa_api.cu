@@ -311,7 +311,8 @@ pisa_status launch_select_tc(const float* qbar, const float* kbar, const float* 
   const size_t smem = SelectTcLayout<D, R>::bytes(ns, nb);
   if (!set_smem(select_sm100_kernel<D, R>, smem)) return PISA_ERR_CUDA;
   const float scale = 1.0f / sqrtf((float)D);
-  select_sm100_kernel<D, R><<<dim3((nb + R - 1) / R, s.BH()), kSelTcThreads, smem, st>>>(
+  const dim3 grid = (nb % R) != 0 ? dim3(s.BH(), (nb + R - 1) / R) : dim3((nb + R - 1) / R, s.BH());
+  select_sm100_kernel<D, R><<<grid, kSelTcThreads, smem, st>>>(
       mK, qbar, M, s.L, s.block, nb, k, ns, scale, sel);
   return last_launch();
 }

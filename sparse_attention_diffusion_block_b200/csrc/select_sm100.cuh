@@ -63,7 +63,10 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Grid (ceil(nb / R), BH), kSelTcThreads threads, dynamic shared memory
+// Grid (BH, ceil(nb / R)) when nb is not a multiple of R (heads fastest: the
+// CTAs of each head's last, partly filled row tile, with a shorter top-k, run
+// last, in the partial wave at the end of the grid), else (ceil(nb / R), BH)
+// (a head's CTAs together).  kSelTcThreads threads, dynamic shared memory
 // SelectTcLayout<D, R>::bytes(ns, nb); ns >= 2 stages.
 // tmK: kbar fp32 [BH][nb][D], boxes of 32 dims x 128 blocks, 128-byte swizzle,
 // rows past nb read as zero.
@@ -101,7 +104,9 @@ select_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const float* __rest
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int bh = blockIdx.y, i0 = blockIdx.x * R;
+  const bool heads_fast = (nb % R) != 0;
+  const int bh = heads_fast ? blockIdx.x : blockIdx.y;
+  const int i0 = (heads_fast ? blockIdx.y : blockIdx.x) * R;
   const int rows = min(R, nb - i0);
   const int ntiles = (nb + 127) / 128;
   const int nit = ntiles * NH;
