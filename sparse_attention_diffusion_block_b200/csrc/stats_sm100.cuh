@@ -379,17 +379,24 @@ cov_norm_sm100_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_cons
       hb[b + 2] = w.z;
       hb[b + 3] = w.w;
     }
+    // this thread's kbar and vsum entries of the next block, loaded one block
+    // ahead so their latency hides behind the current block's epilogue
+    const size_t ob = ((size_t)bh * nb + j0) * D + a;
+    float kb_next = kbar[ob], vs_next = vsum[ob];
     for (int jj = 0; jj < nj; ++jj) {
       const int buf = jj & 1;
       const int j = j0 + jj;
-      const size_t o = ((size_t)bh * nb + j) * D;
-      const float kb = kbar[o + a];
+      const float kb = kb_next, vs = vs_next;
+      if (jj + 1 < nj) {
+        kb_next = kbar[ob + (size_t)(jj + 1) * D];
+        vs_next = vsum[ob + (size_t)(jj + 1) * D];
+      }
       // every thread needs the whole vsum_j: staged in shared memory before
-      // the wait for H_j, so the load's latency hides behind it.  Three
-      // buffers: a thread starting block jj knows every epilogue thread has
-      // finished block jj - 3 (the MMA of jj - 1 waited for d_free of jj - 3).
+      // the wait for H_j.  Three buffers: a thread starting block jj knows
+      // every epilogue thread has finished block jj - 3 (the MMA of jj - 1
+      // waited for d_free of jj - 3).
       const int vb = jj % 3;
-      sig[vb * D + a] = vsum[o + a];
+      sig[vb * D + a] = vs;
       mbar_arrive(&vs_full[vb]);
       const float4* s4 = reinterpret_cast<const float4*>(sig + vb * D);
       if (!__all_sync(0xffffffffu, mbar_wait(&d_full[buf], (jj >> 1) & 1, abort))) break;
